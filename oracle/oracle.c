@@ -1,0 +1,478 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU reference of one draft-tree verification step
+ * (EAGLE / EAGLE-2 speculative sampling).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library.  It shares no code with the
+ * CUDA path: its own input decoding, its own Philox, its own walk.
+ *
+ * What it computes, and where the pages define it ("EAGLE: Speculative Sampling
+ * Requires Rethinking Feature Uncertainty", paperlayer.ai summary, abbreviated
+ * "EAGLE summary" below):
+ *
+ *   O1 tree attention   (EAGLE summary, section 3 "Drafting and verification" and
+ *                        "Training and verification": the target verifies the tree
+ *                        in one pass with tree attention): every node i attends to
+ *                        the prefix plus its own ancestors and itself, nothing else.
+ *   O2 LM-head logits   (EAGLE summary, section 3 "Draft model": the LM head turns
+ *                        features into token distributions): logits = hidden W^T.
+ *   O3 accept/resample  (EAGLE summary, section 2 "Preliminaries": accept a drafted
+ *                        token with probability min(1, p(t)/p_hat(t)); after a
+ *                        rejection the rest of that draft is discarded and a token
+ *                        is resampled; appendix A.2 "Multi-Round Speculative
+ *                        Sampling": the rule is applied recursively over the k
+ *                        candidates of a tree node, and sampling falls back to an
+ *                        adjusted distribution; appendix B: Algorithm 1 takes the
+ *                        target distribution, the candidates and their own
+ *                        distributions and returns one sample of the target).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - the adjusted distribution is norm(max(0, p - p_hat)) (standard speculative
+ *     sampling residual); if its mass is 0 the previous p is kept;
+ *   - candidates are tried in ascending node index; p is updated after each
+ *     rejection and the next candidate is tested against the updated p;
+ *   - p_hat(t) == 0 accepts (the ratio is +inf);
+ *   - temperature T: p = softmax(logits / T); T == 0 is greedy argmax matching
+ *     (EAGLE summary, section 4: "temperature=0"; EAGLE-2 blog, section 1: T = 0
+ *     always takes the most probable token), ties to the lowest token index;
+ *   - when the walk ends it emits one more token: the argmax (T == 0), or a sample
+ *     of the current p -- the residual after the last rejection, else the
+ *     unadjusted p at the final node;
+ *   - sampling is the exponential race: argmin over v with p_v > 0 of E_v / p_v,
+ *     E_v = -ln U_v, lowest v on ties;
+ *   - uniforms are Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
+ *     numbers: as easy as 1, 2, 3", SC'11) with key = seed and counter
+ *     (v >> 2, b << 16 | purpose << 8 | node, offset_lo, offset_hi); word v & 3;
+ *     U = (2 * (x >> 9) + 1) * 2^-24.  The accept test of candidate c uses
+ *     (node c, v 0, purpose 0); the race at node n uses (node n, v, purpose 1).
+ *
+ * Parity pins live in the not-gpu tests: brute-force path attention and torch's
+ * causal SDPA in float64 (O1), numpy float64 matmul (O2), brute-force argmax path
+ * matching at T = 0 and chi-square tests of the emitted-token distribution, the
+ * closed-form single-candidate acceptance probability and the race sampler (O3).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_F32 0
+#define ORC_BF16 1
+
+#define ORC_OK 0
+#define ORC_BAD_TREE 1
+#define ORC_BAD_ARG 2
+
+/* ------------------------------------------------------------------ input decoding */
+
+static inline double orc_ld(const void *base, size_t i, int elem_type)
+{
+    if (elem_type == ORC_BF16) {
+        uint32_t bits = (uint32_t)((const uint16_t *)base)[i] << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)base)[i];
+}
+
+/* ------------------------------------------------------------------ Philox4x32-10 */
+
+/* One Philox round: two 32x32->64 products, the high halves mixed with the other
+ * two counter words and the key (Salmon et al. SC'11, section 3.2). */
+static void orc_philox_round(uint32_t c[4], const uint32_t k[2])
+{
+    const uint64_t prod0 = (uint64_t)0xD2511F53u * c[0];
+    const uint64_t prod1 = (uint64_t)0xCD9E8D57u * c[2];
+    const uint32_t hi0 = (uint32_t)(prod0 >> 32), lo0 = (uint32_t)prod0;
+    const uint32_t hi1 = (uint32_t)(prod1 >> 32), lo1 = (uint32_t)prod1;
+    const uint32_t n0 = hi1 ^ c[1] ^ k[0];
+    const uint32_t n2 = hi0 ^ c[3] ^ k[1];
+    c[0] = n0;
+    c[1] = lo1;
+    c[2] = n2;
+    c[3] = lo0;
+}
+
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+    uint32_t k[2] = {key[0], key[1]};
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) { /* Weyl key schedule between rounds */
+            k[0] += 0x9E3779B9u;
+            k[1] += 0xBB67AE85u;
+        }
+        orc_philox_round(c, k);
+    }
+    memcpy(out, c, sizeof c);
+}
+
+double orc_uniform(uint64_t seed, uint64_t offset, int32_t b, int32_t node, int32_t v,
+                   int32_t purpose)
+{
+    const uint32_t ctr[4] = {(uint32_t)v >> 2,
+                             ((uint32_t)b << 16) | ((uint32_t)purpose << 8) | (uint32_t)node,
+                             (uint32_t)offset, (uint32_t)(offset >> 32)};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    orc_philox4x32_10(ctr, key, w);
+    const uint32_t x = w[v & 3];
+    return (2.0 * (double)(x >> 9) + 1.0) * ldexp(1.0, -24);
+}
+
+/* ------------------------------------------------------------------ tree */
+
+/* A valid tree is topologically ordered: parent[0] = -1, 0 <= parent[i] < i. */
+int orc_check_tree(int32_t N, const int32_t *parents)
+{
+    if (N < 1 || N > 64 || parents[0] != -1) return ORC_BAD_TREE;
+    for (int i = 1; i < N; ++i)
+        if (parents[i] < 0 || parents[i] >= i) return ORC_BAD_TREE;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ O1 attention */
+
+/* out[b,i,h] = sum_j softmax_j(scale * q[b,i,h] . k_j) v_j, with j over the prefix
+ * positions 0..L_b-1 of kv head h / (Hq/Hkv), then the tree nodes on the path from
+ * node i up to the root (node i itself included). */
+static void orc_attention_row(int b, int i, int h, int N, int Hq, int Hkv, int D, int Lmax,
+                              int et, const void *q, const void *kp, const void *vp,
+                              const int32_t *prefix_lens, const void *kt, const void *vt,
+                              const int32_t *parents, double scale, double *out_row,
+                              double *scores)
+{
+    const int G = Hq / Hkv;
+    const int g = h / G;
+    const int L = prefix_lens[b];
+    const size_t qoff = (((size_t)b * N + i) * Hq + h) * (size_t)D;
+    int path[64];
+    int np = 0;
+    for (int a = i; a >= 0; a = parents[(size_t)b * N + a]) path[np++] = a;
+
+    const int nk = L + np;
+    double mx = -INFINITY;
+    for (int j = 0; j < nk; ++j) {
+        size_t koff;
+        const void *ksrc;
+        if (j < L) {
+            koff = (((size_t)b * Hkv + g) * Lmax + j) * (size_t)D;
+            ksrc = kp;
+        } else {
+            koff = (((size_t)b * N + path[j - L]) * Hkv + g) * (size_t)D;
+            ksrc = kt;
+        }
+        double s = 0.0;
+        for (int d = 0; d < D; ++d) s += orc_ld(q, qoff + d, et) * orc_ld(ksrc, koff + d, et);
+        s *= scale;
+        scores[j] = s;
+        if (s > mx) mx = s;
+    }
+    double den = 0.0;
+    for (int j = 0; j < nk; ++j) {
+        scores[j] = exp(scores[j] - mx);
+        den += scores[j];
+    }
+    for (int d = 0; d < D; ++d) out_row[d] = 0.0;
+    for (int j = 0; j < nk; ++j) {
+        size_t voff;
+        const void *vsrc;
+        if (j < L) {
+            voff = (((size_t)b * Hkv + g) * Lmax + j) * (size_t)D;
+            vsrc = vp;
+        } else {
+            voff = (((size_t)b * N + path[j - L]) * Hkv + g) * (size_t)D;
+            vsrc = vt;
+        }
+        const double wgt = scores[j] / den;
+        for (int d = 0; d < D; ++d) out_row[d] += wgt * orc_ld(vsrc, voff + d, et);
+    }
+}
+
+/* rows: n_rows triples (b, i, h); NULL means every row in [B, N, Hq] order.
+ * out: [n_rows, D] (or [B*N*Hq, D]).  Returns ORC_BAD_TREE if any sequence's
+ * parents are not a valid tree, ORC_BAD_ARG for bad shapes. */
+int orc_tree_attention(int B, int N, int Hq, int Hkv, int D, int Lmax, int elem_type,
+                       const void *q, const void *k_prefix, const void *v_prefix,
+                       const int32_t *prefix_lens, const void *k_tree, const void *v_tree,
+                       const int32_t *parents, double scale, int n_rows, const int32_t *rows,
+                       double *out)
+{
+    if (B < 1 || N < 1 || N > 64 || Hq < 1 || Hkv < 1 || Hq % Hkv || D < 1 || Lmax < 0)
+        return ORC_BAD_ARG;
+    for (int b = 0; b < B; ++b) {
+        if (orc_check_tree(N, parents + (size_t)b * N) != ORC_OK) return ORC_BAD_TREE;
+        if (prefix_lens[b] < 0 || prefix_lens[b] > Lmax) return ORC_BAD_ARG;
+    }
+    const long total = rows ? n_rows : (long)B * N * Hq;
+#pragma omp parallel
+    {
+        double *scores = (double *)malloc(sizeof(double) * (size_t)(Lmax + 64));
+#pragma omp for schedule(dynamic, 4)
+        for (long r = 0; r < total; ++r) {
+            int b, i, h;
+            if (rows) {
+                b = rows[3 * r];
+                i = rows[3 * r + 1];
+                h = rows[3 * r + 2];
+            } else {
+                b = (int)(r / ((long)N * Hq));
+                i = (int)((r / Hq) % N);
+                h = (int)(r % Hq);
+            }
+            orc_attention_row(b, i, h, N, Hq, Hkv, D, Lmax, elem_type, q, k_prefix, v_prefix,
+                              prefix_lens, k_tree, v_tree, parents, scale,
+                              out + (size_t)r * D, scores);
+        }
+        free(scores);
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ O2 LM head */
+
+static void orc_logits_row(int H, int V, int et, const void *hidden, const void *w, int row,
+                           double *out)
+{
+#pragma omp parallel for schedule(static) if (!omp_in_parallel() && (long)V * H > (1L << 20))
+    for (int v = 0; v < V; ++v) {
+        double s = 0.0;
+        const size_t ho = (size_t)row * H, wo = (size_t)v * H;
+        for (int k = 0; k < H; ++k) s += orc_ld(hidden, ho + k, et) * orc_ld(w, wo + k, et);
+        out[v] = s;
+    }
+}
+
+/* logits[r, v] = sum_k hidden[row_r, k] * W[v, k]; rows NULL = all M rows. */
+void orc_lm_head(int M, int H, int V, int elem_type, const void *hidden, const void *w,
+                 int n_rows, const int32_t *rows, double *logits)
+{
+    const int nr = rows ? n_rows : M;
+    if ((long)nr * V >= 4096 && nr > 1) {
+#pragma omp parallel for collapse(2) schedule(static)
+        for (int r = 0; r < nr; ++r)
+            for (int v = 0; v < V; ++v) {
+                const int row = rows ? rows[r] : r;
+                double s = 0.0;
+                const size_t ho = (size_t)row * H, wo = (size_t)v * H;
+                for (int k = 0; k < H; ++k)
+                    s += orc_ld(hidden, ho + k, elem_type) * orc_ld(w, wo + k, elem_type);
+                logits[(size_t)r * V + v] = s;
+            }
+    } else {
+        for (int r = 0; r < nr; ++r)
+            orc_logits_row(H, V, elem_type, hidden, w, rows ? rows[r] : r,
+                           logits + (size_t)r * V);
+    }
+}
+
+/* ------------------------------------------------------------------ O3 accept / resample */
+
+/* Exponential race: argmin over v with weight_v > 0 of (-ln U(b, node, v, 1)) / weight_v,
+ * lowest v on ties.  *rel_gap receives (second - best) / best, or +inf if only one
+ * candidate. */
+int32_t orc_race(int V, const double *weight, uint64_t seed, uint64_t offset, int32_t b,
+                 int32_t node, double *rel_gap)
+{
+    double best = INFINITY, second = INFINITY;
+    int32_t arg = -1;
+    for (int v = 0; v < V; ++v) {
+        if (!(weight[v] > 0.0)) continue;
+        const double e = -log(orc_uniform(seed, offset, b, node, v, 1));
+        const double key = e / weight[v];
+        if (key < best) {
+            second = best;
+            best = key;
+            arg = v;
+        } else if (key < second) {
+            second = key;
+        }
+    }
+    if (rel_gap) *rel_gap = (arg >= 0 && isfinite(second)) ? (second - best) / best : INFINITY;
+    return arg;
+}
+
+typedef struct {
+    int mode; /* 0: float logits array, 1: double logits array, 2: hidden x W on demand */
+    const void *logits;
+    int N, V, H, elem_type;
+    const void *hidden, *w;
+} orc_rows_t;
+
+static void orc_get_row(const orc_rows_t *src, int b, int node, double *row)
+{
+    const size_t base = ((size_t)b * src->N + node) * (size_t)src->V;
+    if (src->mode == 0) {
+        for (int v = 0; v < src->V; ++v) row[v] = ((const float *)src->logits)[base + v];
+    } else if (src->mode == 1) {
+        memcpy(row, (const double *)src->logits + base, sizeof(double) * (size_t)src->V);
+    } else {
+        orc_logits_row(src->H, src->V, src->elem_type, src->hidden, src->w, b * src->N + node,
+                       row);
+    }
+}
+
+typedef struct {
+    int32_t near;     /* decisions within the margin */
+    int32_t decisions;
+    int32_t first_near; /* index of the first near decision, -1 if none */
+} orc_diag_t;
+
+static void orc_note(orc_diag_t *dg, int is_near)
+{
+    if (is_near) {
+        if (dg->near == 0) dg->first_near = dg->decisions;
+        dg->near++;
+    }
+    dg->decisions++;
+}
+
+/* One sequence of the multi-round speculative sampling walk.  Returns the number of
+ * accepted drafted nodes (written to acc[]), or -1 for an invalid tree. */
+static int orc_walk(const orc_rows_t *src, int b, int N, int V, const float *draft_b,
+                    const int32_t *tokens_b, const int32_t *parents_b, double T, uint64_t seed,
+                    uint64_t offset, double margin, int32_t *acc, int32_t *next_token,
+                    orc_diag_t *dg, double *logit_row, double *p, double *r)
+{
+    if (orc_check_tree(N, parents_b) != ORC_OK) return -1;
+    for (int i = 1; i < N; ++i)
+        if (tokens_b[i] < 0 || tokens_b[i] >= V) return -1;
+
+    int n_acc = 0;
+    int cur = 0; /* the committed root */
+    for (;;) {
+        orc_get_row(src, b, cur, logit_row);
+        if (T == 0.0) {
+            /* greedy: the target's choice is argmax(logits), lowest index on ties */
+            int m = 0;
+            for (int v = 1; v < V; ++v)
+                if (logit_row[v] > logit_row[m]) m = v;
+            double second = -INFINITY;
+            for (int v = 0; v < V; ++v)
+                if (v != m && logit_row[v] > second) second = logit_row[v];
+            orc_note(dg, V > 1 && logit_row[m] - second <= margin);
+            int matched = -1;
+            for (int c = cur + 1; c < N; ++c)
+                if (parents_b[c] == cur && tokens_b[c] == m) {
+                    matched = c;
+                    break;
+                }
+            if (matched >= 0) {
+                acc[n_acc++] = matched;
+                cur = matched;
+                continue;
+            }
+            *next_token = m;
+            return n_acc;
+        }
+
+        /* p = softmax(logits / T) */
+        double mx = -INFINITY;
+        for (int v = 0; v < V; ++v)
+            if (logit_row[v] / T > mx) mx = logit_row[v] / T;
+        double z = 0.0;
+        for (int v = 0; v < V; ++v) {
+            p[v] = exp(logit_row[v] / T - mx);
+            z += p[v];
+        }
+        for (int v = 0; v < V; ++v) p[v] /= z;
+
+        int accepted = -1;
+        for (int c = cur + 1; c < N && accepted < 0; ++c) {
+            if (parents_b[c] != cur) continue;
+            const int t_hat = tokens_b[c];
+            const float *p_hat = draft_b + (size_t)c * V;
+            const double u = orc_uniform(seed, offset, b, c, 0, 0);
+            if (p_hat[t_hat] == 0.0f) {
+                orc_note(dg, 0);
+                accepted = c;
+                break;
+            }
+            const double ratio = p[t_hat] / (double)p_hat[t_hat];
+            orc_note(dg, fabs(u - ratio) <= margin * (ratio > 1.0 ? ratio : 1.0));
+            if (u < ratio) {
+                accepted = c;
+                break;
+            }
+            /* rejected: p <- norm(max(0, p - p_hat)) */
+            double mass = 0.0;
+            for (int v = 0; v < V; ++v) {
+                const double d = p[v] - (double)p_hat[v];
+                r[v] = d > 0.0 ? d : 0.0;
+                mass += r[v];
+            }
+            if (mass > 0.0)
+                for (int v = 0; v < V; ++v) p[v] = r[v] / mass;
+        }
+        if (accepted >= 0) {
+            acc[n_acc++] = accepted;
+            cur = accepted;
+            continue;
+        }
+        double gap;
+        *next_token = orc_race(V, p, seed, offset, b, cur, &gap);
+        orc_note(dg, gap <= margin);
+        return n_acc;
+    }
+}
+
+/* logits_mode 0: `logits` is float [B,N,V]; 1: double [B,N,V]; 2: rows are computed on
+ * demand from hidden [B*N,H] and w [V,H] (elem_type).  Outputs: accepted_nodes [B,N]
+ * (-1 padded), accept_len [B] and next_token [B] (-1 and -1 for an invalid tree);
+ * diagnostics (may be NULL): near_count, n_decisions, first_near per sequence. */
+int orc_tree_accept(int B, int N, int V, int logits_mode, const void *logits, int H,
+                    int elem_type, const void *hidden, const void *w, const float *draft_probs,
+                    const int32_t *tokens, const int32_t *parents, double temperature,
+                    uint64_t seed, uint64_t offset, double margin, int32_t *accepted_nodes,
+                    int32_t *accept_len, int32_t *next_token, int32_t *near_count,
+                    int32_t *n_decisions, int32_t *first_near)
+{
+    if (B < 1 || B > 65535 || N < 1 || N > 64 || V < 1 || !(temperature >= 0.0))
+        return ORC_BAD_ARG;
+    const orc_rows_t src = {logits_mode, logits, N, V, H, elem_type, hidden, w};
+#pragma omp parallel if (B > 16 && logits_mode != 2)
+    {
+        double *row = (double *)malloc(sizeof(double) * (size_t)V);
+        double *p = (double *)malloc(sizeof(double) * (size_t)V);
+        double *r = (double *)malloc(sizeof(double) * (size_t)V);
+#pragma omp for schedule(dynamic, 64)
+        for (int b = 0; b < B; ++b) {
+            int32_t *acc = accepted_nodes + (size_t)b * N;
+            for (int i = 0; i < N; ++i) acc[i] = -1;
+            orc_diag_t dg = {0, 0, -1};
+            int32_t nt = -1;
+            const int n = orc_walk(&src, b, N, V, draft_probs + (size_t)b * N * V,
+                                   tokens + (size_t)b * N, parents + (size_t)b * N,
+                                   temperature, seed, offset, margin, acc, &nt, &dg, row, p, r);
+            accept_len[b] = n;
+            next_token[b] = n < 0 ? -1 : nt;
+            if (near_count) near_count[b] = dg.near;
+            if (n_decisions) n_decisions[b] = dg.decisions;
+            if (first_near) first_near[b] = dg.first_near;
+        }
+        free(row);
+        free(p);
+        free(r);
+    }
+    return ORC_OK;
+}
+
+/* Uniforms U(b, node, v, purpose) for v = 0..n-1 (test helper for the generator pins). */
+void orc_fill_uniforms(uint64_t seed, uint64_t offset, int32_t b, int32_t node, int32_t purpose,
+                       int32_t n, double *out)
+{
+    for (int32_t v = 0; v < n; ++v) out[v] = orc_uniform(seed, offset, b, node, v, purpose);
+}
+
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

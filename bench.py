@@ -1,0 +1,333 @@
+"""Benchmark of one draft-tree verification step (tree attention + LM-head logits + the
+accept/resample walk) on B200, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--temperature T]
+
+Default workload: the Vicuna-7B-shaped static EAGLE tree (batch 1, 32 heads, head_dim 128,
+bf16, prefix 1024, 45 tree rows, hidden 4096, vocab 32000) at temperature 1.  The batch-1
+step does not shard, so N GPUs run N independent replicas ("scaling": "weak"); the value
+is all replicas' steps over the slowest rank's device time.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (fp64, all host cores) on a bounded sample of the
+same workload; it is a reported baseline, not a tuned program.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "tree-verify steps/s and tree-tokens/s at 1 B200; achieved HBM GB/s as % of peak"
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def step_bytes(w, prefix_lens):
+    el = 2 if w.dtype == wl.BF16 else 4
+    B, N, Hq, Hkv, D, H, V = (w.batch, w.num_nodes, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                              w.hidden, w.vocab)
+    kv = int(np.sum(prefix_lens)) * Hkv * D * 2 * el
+    wbytes = V * H * el
+    lm = wbytes + B * N * H * el + B * N * V * 4
+    return dict(kv=kv, w=wbytes, lm_head=lm, roofline_bytes=kv + wbytes)
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle (CPU baseline)
+
+def oracle_step_sample(w, inp, T, lm_stride=8):
+    """One oracle step on a bounded sample: attention for every row, LM-head logits for
+    every `lm_stride`-th tree row, and the full accept walk (which computes the logits
+    rows it visits).  Returns the extrapolated seconds of one whole step and a label."""
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.tree_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["prefix_lens"],
+                          inp["k_tree"], inp["v_tree"], inp["parents"])
+    t1 = time.perf_counter()
+    M = w.batch * w.num_nodes
+    rows = np.arange(0, M, lm_stride, dtype=np.int32)
+    oracle.lm_head(inp["hidden"], inp["w_lm"], rows=rows)
+    t2 = time.perf_counter()
+    oracle.tree_accept(inp["draft_probs"], inp["tokens"], inp["parents"], T,
+                       hidden=inp["hidden"], w_lm=inp["w_lm"])
+    t3 = time.perf_counter()
+    full = (t1 - t0) + (t2 - t1) * M / len(rows) + (t3 - t2)
+    label = (f"attention all {w.batch * w.num_nodes * w.num_q_heads} rows + LM head {len(rows)} of "
+             f"{M} rows (scaled x{M / len(rows):.2f}) + full accept walk; fp64 C oracle")
+    return full, label, oracle.num_threads()
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="vicuna7b_static", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--temperature", type=float, default=1.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = wl.WORKLOADS[args.workload]
+    T = args.temperature
+    config = {"workload": f"{w.name}: B{w.batch} Hq{w.num_q_heads}/Hkv{w.num_kv_heads} D{w.head_dim} "
+                          f"{w.dtype} prefix {w.prefix_len if w.prefix_min is None else f'U[{w.prefix_min},{w.prefix_len}]'} "
+                          f"N{w.num_nodes} H{w.hidden} V{w.vocab} T{T:g}",
+              "batch": w.batch, "tree_nodes": w.num_nodes, "prefix_len": w.prefix_len,
+              "hidden": w.hidden, "vocab": w.vocab, "temperature": T,
+              "l2": "flushed before every step (512 MiB write, untimed)",
+              "parallelism": "replicas" if world > 1 else "single"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inp = wl.generate(w, T)
+        times = []
+        label, cores = "", 1
+        for i in range(args.steps + args.warmup):
+            t, label, cores = oracle_step_sample(w, inp, T)
+            if i >= args.warmup:
+                times.append(t)
+        sec = float(np.mean(times))
+        value = 1.0 / sec
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "verify-steps/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config,
+            "tree_tokens_per_s": value * w.batch * w.num_nodes,
+            "cpu_baseline": {"value": value, "unit": "verify-steps/s", "cores": cores,
+                             "kind": "oracle", "sample": label},
+            "e2e": {"value": value, "unit": "verify-steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return
+
+    import torch
+    from tree_verify_b200 import binding
+    from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    binding.load()
+
+    inp = wl.generate(w, T, seed=None)
+    shape = shape_from_workload(w)
+    x = StepInputs.from_numpy(inp, w.dtype, device=dev)
+    step = VerifyStep(shape, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nb = step_bytes(w, inp["prefix_lens"])
+    # kernels this library launches per step: attention (+ split merge), LM head, walk
+    attn_splits = binding.workspace_bytes(shape) > 0
+    launches_per_step = 3 + (1 if attn_splits else 0)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # warm-up (also lets the clocks ramp)
+    for i in range(args.warmup):
+        flush.zero_()
+        step.run(x, T, seed=rank, offset=i)
+    t_end = time.time() + 0.5
+    while time.time() < t_end:
+        flush.zero_()
+        step.run(x, T, seed=rank, offset=0)
+    barrier()
+    assert binding.device_error(reset=True) == 0
+
+    # ---- timed region: K whole steps through eagle_verify_step, L2 flushed before each
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step.run(x, T, seed=rank, offset=i)
+            ends[i].record(stream)
+        barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(np.sum(step_ms))
+
+    # ---- dominant kernel alone (LM head), same conditions, for the roofline
+    ls = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    le = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        ls[i].record(stream)
+        step.lm_head(x)
+        le[i].record(stream)
+    barrier()
+    lm_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(ls, le)]))
+
+    # ---- end to end through the public API with host buffers: per-step tree inputs
+    # (queries, tree K/V, hidden states, parents, tokens, draft distributions) copied from
+    # pinned host memory, the walk's results read back; the prefix K/V cache and W stay
+    # resident as model state.
+    per_step = ["q", "k_tree", "v_tree", "hidden", "parents", "tokens", "draft_probs", "prefix_lens"]
+    host = {n: getattr(x, n).cpu().pin_memory() for n in per_step}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    out_host = [torch.empty_like(t, device="cpu").pin_memory()
+                for t in (step.accepted_nodes, step.accept_len, step.next_token)]
+    d2h = sum(t.numel() * t.element_size() for t in out_host)
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        es[i].record(stream)
+        for n in per_step:
+            getattr(x, n).copy_(host[n], non_blocking=True)
+        step.run(x, T, seed=rank, offset=i)
+        for dst, src in zip(out_host, (step.accepted_nodes, step.accept_len, step.next_token)):
+            dst.copy_(src, non_blocking=True)
+        ee[i].record(stream)
+    barrier()
+    e2e_ms = float(np.sum([s.elapsed_time(e) for s, e in zip(es, ee)]))
+    assert binding.device_error(reset=True) == 0
+
+    # ---- max over ranks
+    t = torch.tensor([total_ms, e2e_ms, lm_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, lm_ms = (float(v) for v in t.tolist())
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    value = world * args.steps / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+    peak, peak_kind = _peaks()
+    lm_gbs = nb["lm_head"] / (lm_ms / 1e3) / 1e9
+    step_gbs = nb["roofline_bytes"] / (ms_per_step / 1e3) / 1e9
+    result = {
+        "metric": METRIC, "value": value, "unit": "verify-steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic", "config": config,
+        "tree_tokens_per_s": value * w.batch * w.num_nodes,
+        "step_hbm_gbs": step_gbs,
+        "step_roofline_frac": step_gbs / peak,
+        "step_roofline_note": f"(KV + W bytes) / step time vs {peak_kind} HBM {peak:.0f} GB/s; "
+                              f"(KV + W) = {nb['roofline_bytes']} B",
+        "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
+        "roofline": {"kernel": "lm_head_tc_kernel", "bound": "hbm", "achieved": lm_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": lm_gbs / peak,
+                     "traffic": None, "bytes_per_launch": nb["lm_head"],
+                     "us_per_launch": lm_ms * 1e3, "peak_kind": peak_kind},
+        "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "verify-steps/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline:
+        # about 10-30 s of oracle work: repeat the bounded sample, report the mean
+        secs, t0 = [], time.perf_counter()
+        while not secs or (time.perf_counter() - t0 < 10.0 and len(secs) < 50):
+            sec, label, cores = oracle_step_sample(w, inp, T)
+            secs.append(sec)
+        result["cpu_baseline"] = {"value": 1.0 / float(np.mean(secs)), "unit": "verify-steps/s",
+                                  "cores": cores, "kind": "oracle",
+                                  "sample": f"{len(secs)} x [{label}]"}
+    print(json.dumps(result))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

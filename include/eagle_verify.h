@@ -1,0 +1,175 @@
+/*
+ * eagle_verify.h -- C ABI of the B200 (sm_100a) draft-tree verification library.
+ *
+ * One verification pass of EAGLE / EAGLE-2 speculative sampling ("EAGLE:
+ * Speculative Sampling Requires Rethinking Feature Uncertainty", paperlayer.ai
+ * summary, called "EAGLE summary" below; the EAGLE-2 blog post republished at
+ * m.jxzklqfsx.com, called "EAGLE-2 blog"): the target model scores every node of
+ * a drafted token tree in one pass, and the accept/resample rule walks the tree.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, dense, row-major, 16-byte aligned.
+ *     The caller owns every buffer; the library never allocates or frees memory.
+ *     Scratch memory comes only from the caller's `workspace` (size from
+ *     eagle_workspace_bytes()).
+ *   - `stream` is a cudaStream_t passed as void*.  Every call is asynchronous on it:
+ *     nothing is synchronised and no device data is read on the host.
+ *   - Errors the host can see (shapes, null or misaligned pointers, N > 64,
+ *     Hq % Hkv != 0, T < 0, workspace too small) return a status before anything
+ *     is enqueued.  A CUDA launch failure returns EAGLE_ERR_CUDA.
+ *   - Errors only the device can see (a malformed tree or an out-of-range token in
+ *     `parents`/`tokens`) never trap: eagle_tree_accept writes accept_len = -1 and
+ *     next_token = -1 for that sequence; tree attention then treats an invalid
+ *     parent link as "no ancestors" for that node and still writes finite output.
+ *   - Device-side waits are bounded.  If one gives up (a hardware stall, never a
+ *     normal run) the kernel records a code readable with eagle_device_error().
+ *   - No C++ exception crosses this boundary.
+ *
+ * Shape symbols: B batch, N tree rows per sequence (root node 0 included, <= 64),
+ * Hq / Hkv query / key-value heads (G = Hq / Hkv), D head_dim (64 or 128),
+ * Lmax prefix stride, H hidden size, V vocabulary size.
+ */
+#ifndef EAGLE_VERIFY_H
+#define EAGLE_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    EAGLE_OK = 0,
+    EAGLE_ERR_INVALID_ARGUMENT = 1,
+    EAGLE_ERR_UNSUPPORTED = 2,
+    EAGLE_ERR_WORKSPACE_TOO_SMALL = 3,
+    EAGLE_ERR_CUDA = 4
+} eagle_status_t;
+
+typedef enum {
+    EAGLE_DTYPE_F32 = 0,  /* float32 inputs, float32 arithmetic (exactness path) */
+    EAGLE_DTYPE_BF16 = 1  /* bfloat16 inputs, float32 accumulation */
+} eagle_dtype_t;
+
+typedef struct {
+    int32_t batch;          /* B, 1..65535                                           */
+    int32_t num_nodes;      /* N, 1..64, root node 0 included                         */
+    int32_t num_q_heads;    /* Hq                                                     */
+    int32_t num_kv_heads;   /* Hkv; Hq % Hkv == 0                                     */
+    int32_t head_dim;       /* D in {64, 128}                                         */
+    int32_t max_prefix_len; /* Lmax >= 1: row stride (in positions) of prefix K/V     */
+    int32_t hidden;         /* H >= 1 (multiple of 8 for bf16)                         */
+    int32_t vocab;          /* V >= 1                                                 */
+    int32_t dtype;          /* eagle_dtype_t of q, k/v, hidden, w_lm and attention out */
+    float softmax_scale;    /* <= 0 selects 1/sqrt(D)                                  */
+} eagle_shape_t;
+
+/* Human-readable name of a status code (static storage). */
+const char *eagle_status_string(eagle_status_t status);
+
+/* Bytes of `workspace` the entry points below need for this shape (0 if the shape is
+ * invalid).  The split-KV partials of tree attention live there. */
+size_t eagle_workspace_bytes(const eagle_shape_t *shape);
+
+/*
+ * Tree attention (EAGLE summary, section 3 "Drafting and verification" / "Training and
+ * verification": the target verifies the tree-structured draft in one forward pass
+ * with tree attention; appendix A.1 "Tree Structure").  For sequence b, node i and
+ * query head h, with kv head g = h / G:
+ *     out[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k_j) v_j
+ * where j runs over prefix positions 0 .. prefix_lens[b]-1 of kv head g and over the
+ * tree nodes on the path from i to the root, i included.
+ *   q            [B,N,Hq,D]       dtype
+ *   k_prefix     [B,Hkv,Lmax,D]   dtype; positions >= prefix_lens[b] are never read
+ *   v_prefix     [B,Hkv,Lmax,D]   dtype
+ *   prefix_lens  [B] int32, each in 0..Lmax
+ *   k_tree       [B,N,Hkv,D]      dtype; keys of the tree nodes (post-RoPE)
+ *   v_tree       [B,N,Hkv,D]      dtype
+ *   parents      [B,N] int32: parents[b,0] = -1, 0 <= parents[b,i] < i
+ *   out          [B,N,Hq,D]       dtype
+ *   workspace    >= eagle_workspace_bytes(shape) bytes, 256-byte aligned
+ */
+eagle_status_t eagle_tree_attention(const eagle_shape_t *shape, const void *q,
+                                    const void *k_prefix, const void *v_prefix,
+                                    const int32_t *prefix_lens, const void *k_tree,
+                                    const void *v_tree, const int32_t *parents, void *out,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * LM-head logits for every tree node (EAGLE summary, section 3 "Draft model": the LM
+ * head turns features into token probabilities; the target's LM head scores all
+ * tree nodes in the verification pass):
+ *     logits[r, v] = sum_k hidden[r, k] * w_lm[v, k]     (fp32 accumulation)
+ *   hidden  [B*N, H]  dtype
+ *   w_lm    [V, H]    dtype (nn.Linear layout, H contiguous)
+ *   logits  [B*N, V]  float32
+ */
+eagle_status_t eagle_lm_head_logits(const eagle_shape_t *shape, const void *hidden,
+                                    const void *w_lm, float *logits, void *stream);
+
+/*
+ * The accept / resample walk (EAGLE summary, section 2 "Preliminaries": accept a
+ * drafted token t with probability min(1, p(t)/p_hat(t)), discard the rest of that
+ * branch after a rejection and resample; appendix A.2 "Multi-Round Speculative
+ * Sampling" and appendix B "Algorithm 1": the rule is applied over the k candidates
+ * of a node, falling back to an adjusted distribution).  Per sequence, from the root:
+ *   T == 0: greedy -- the first child (ascending index) whose token equals
+ *           argmax(logits[cur]) (lowest index on ties) is accepted; otherwise the walk
+ *           ends and emits that argmax.
+ *   T  > 0: p = softmax(logits[cur] / T); each child c in ascending index is accepted
+ *           when u(b, c) < p(t_c) / p_hat_c(t_c) (or p_hat_c(t_c) == 0); after a
+ *           rejection p <- norm(max(0, p - p_hat_c)) (kept if that mass is 0).  When
+ *           no child is accepted the walk ends and emits a sample of the current p
+ *           (the residual, or the unadjusted p at a leaf).
+ * Uniforms are Philox4x32-10 with key = seed and counter
+ * (v >> 2, b << 16 | purpose << 8 | node, offset_lo, offset_hi), word v & 3,
+ * u = (2 * (x >> 9) + 1) * 2^-24; accept tests use (node c, v 0, purpose 0); the final
+ * sample is the exponential race argmin_v -ln u(b, cur, v, 1) / p_v, lowest v on ties.
+ *   logits          [B,N,V] float32 (the output of eagle_lm_head_logits)
+ *   draft_probs     [B,N,V] float32; row c = the distribution node c was drafted from
+ *                   (row 0 unused); read only for tested candidates
+ *   tokens          [B,N] int32; tokens[b,0] is the committed root token (unused)
+ *   parents         [B,N] int32
+ *   temperature     >= 0
+ *   accepted_nodes  [B,N] int32 out: accepted drafted nodes root-to-leaf, -1 padded
+ *   accept_len      [B] int32 out: number of accepted nodes, -1 for an invalid tree
+ *   next_token      [B] int32 out: the one extra emitted token, -1 for an invalid tree
+ *   workspace       as for eagle_tree_attention (unused today; pass the same buffer)
+ */
+eagle_status_t eagle_tree_accept(const eagle_shape_t *shape, const float *logits,
+                                 const float *draft_probs, const int32_t *tokens,
+                                 const int32_t *parents, float temperature, uint64_t seed,
+                                 uint64_t offset, int32_t *accepted_nodes, int32_t *accept_len,
+                                 int32_t *next_token, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/*
+ * One whole verification step: tree attention, LM-head logits and the accept walk,
+ * enqueued on `stream` (tree attention may run on an internal side stream that joins
+ * `stream` before the call's work completes; the attention output does not feed the
+ * walk).  Arguments as above; writes out, logits, accepted_nodes, accept_len and
+ * next_token.
+ */
+eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
+                                 const void *k_prefix, const void *v_prefix,
+                                 const int32_t *prefix_lens, const void *k_tree,
+                                 const void *v_tree, const int32_t *parents,
+                                 const void *hidden, const void *w_lm,
+                                 const float *draft_probs, const int32_t *tokens,
+                                 float temperature, uint64_t seed, uint64_t offset, void *out,
+                                 float *logits, int32_t *accepted_nodes, int32_t *accept_len,
+                                 int32_t *next_token, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/*
+ * Reads (and, if `reset` != 0, clears) the device error word that bounded waits set
+ * when they give up.  Synchronises the current device.  *code = 0 means no error.
+ */
+eagle_status_t eagle_device_error(int32_t *code, int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EAGLE_VERIFY_H */

@@ -1,0 +1,78 @@
+"""Full-size verification steps (the five workload shapes) through eagle_verify_step, in
+the launch configuration the benchmark times, checked against the oracle on sampled
+outputs: attention rows and logits rows it recomputes one by one, and the whole accept
+walk, whose visited logits rows the oracle computes itself in fp64 from hidden and W."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from tests.parity import MARGIN, TOL, compare_accept, row_rel_err
+
+pytestmark = pytest.mark.gpu
+
+CASES = [("tiny_chain", 1.0), ("vicuna7b_static", 0.0), ("vicuna7b_static", 1.0),
+         ("llama70b_dyn", 1.0), ("batched7b", 1.0), ("llama3_8b", 0.0), ("llama3_8b", 1.0)]
+
+
+@pytest.mark.parametrize("name,T", CASES, ids=[f"{n}-T{t:g}" for n, t in CASES])
+def test_verify_step_full_size(cuda_lib, orc, name, T):
+    from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
+    w = wl.WORKLOADS[name]
+    inp = wl.generate(w, T)
+    shape = shape_from_workload(w)
+    x = StepInputs.from_numpy(inp, w.dtype)
+    step = VerifyStep(shape)
+    seed, offset = 0, 0
+    step.run(x, T, seed, offset)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error(reset=True) == 0
+    B, N = w.batch, w.num_nodes
+    rng = np.random.default_rng(5)
+
+    # attention: sampled rows (all rows for the tiny case)
+    out = step.out.float().cpu().numpy()
+    if B * N * w.num_q_heads <= 4096:
+        ref = orc.tree_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["prefix_lens"],
+                                 inp["k_tree"], inp["v_tree"], inp["parents"])
+        err = row_rel_err(out.reshape(-1, w.head_dim), ref.reshape(-1, w.head_dim))
+    else:
+        rows = np.stack([rng.integers(0, B, 256), rng.integers(0, N, 256),
+                         rng.integers(0, w.num_q_heads, 256)], 1).astype(np.int32)
+        rows[0] = [B - 1, N - 1, w.num_q_heads - 1]
+        ref = orc.tree_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["prefix_lens"],
+                                 inp["k_tree"], inp["v_tree"], inp["parents"], rows=rows)
+        err = row_rel_err(out[rows[:, 0], rows[:, 1], rows[:, 2]], ref)
+    assert err.max() <= TOL[w.dtype], f"attention max row error {err.max():.3e}"
+
+    # logits: sampled rows
+    logits = step.logits.cpu().numpy()
+    lrows = np.unique(np.array([0, B * N - 1, int(rng.integers(0, B * N))], np.int32))
+    lref = orc.lm_head(inp["hidden"], inp["w_lm"], rows=lrows)
+    lerr = row_rel_err(logits[lrows], lref)
+    assert lerr.max() <= TOL[w.dtype], f"logits max row error {lerr.max():.3e}"
+
+    # the walk, against the oracle walking on its own fp64 logits
+    ref_acc = orc.tree_accept(inp["draft_probs"], inp["tokens"], inp["parents"], T, seed=seed,
+                              offset=offset, hidden=inp["hidden"], w_lm=inp["w_lm"], margin=MARGIN)
+    got = dict(accepted_nodes=step.accepted_nodes.cpu().numpy(),
+               accept_len=step.accept_len.cpu().numpy(), next_token=step.next_token.cpu().numpy())
+    exact = compare_accept(got, ref_acc, inp["parents"])
+    assert exact >= B - max(1, B // 8), f"only {exact}/{B} sequences compared exactly"
+
+
+def test_verify_step_stages_equal_fused_call(cuda_lib):
+    """The three stage entry points in sequence give the same bits as eagle_verify_step."""
+    from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
+    w = wl.scaled(wl.WORKLOADS["batched7b"], batch=3, prefix_len=700, prefix_min=100, vocab=5000,
+                  hidden=1024)
+    inp = wl.generate(w, 1.0)
+    x = StepInputs.from_numpy(inp, w.dtype)
+    a, b = VerifyStep(shape_from_workload(w)), VerifyStep(shape_from_workload(w))
+    a.run(x, 1.0, 11, 12)
+    b.attention(x)
+    b.lm_head(x)
+    b.accept(x, 1.0, 11, 12)
+    torch.cuda.synchronize()
+    for name in ("out", "logits", "accepted_nodes", "accept_len", "next_token"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name

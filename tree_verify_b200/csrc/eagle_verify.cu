@@ -1,0 +1,495 @@
+// eagle_verify.cu -- C ABI of the draft-tree verification library (declared in
+// include/eagle_verify.h): argument validation, launch planning, TMA descriptor encoding
+// and the launches of the tree-attention, LM-head and accept kernels.
+//
+// Everything the host can check is checked before anything is enqueued; no entry point
+// allocates memory or synchronises the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/eagle_verify.h"
+#include "accept.cuh"
+#include "attention.cuh"
+#include "device_common.cuh"
+#include "lm_head.cuh"
+
+namespace eagle {
+namespace {
+
+constexpr int kNumSMs = 148;            // B200; launch planning targets this count
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ validation
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+eagle_status_t check_shape(const eagle_shape_t* s) {
+  if (s == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->batch < 1 || s->batch > 65535) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->num_nodes < 1 || s->num_nodes > 64) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->num_q_heads < 1 || s->num_kv_heads < 1 || s->num_q_heads % s->num_kv_heads != 0)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->head_dim != 64 && s->head_dim != 128) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->max_prefix_len < 1) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->hidden < 1 || s->vocab < 1) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->dtype != EAGLE_DTYPE_F32 && s->dtype != EAGLE_DTYPE_BF16) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->dtype == EAGLE_DTYPE_BF16 && s->hidden % 8 != 0) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(s->softmax_scale)) return EAGLE_ERR_INVALID_ARGUMENT;
+  return EAGLE_OK;
+}
+
+float softmax_scale(const eagle_shape_t* s) {
+  return s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / std::sqrt(static_cast<float>(s->head_dim));
+}
+
+// ------------------------------------------------------------------ planning
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct AttnPlan {
+  int row_blocks;
+  int splits;
+  int tiles_per_split;
+  size_t acc_bytes;  // split partials (0 with a single split)
+  size_t ml_bytes;
+};
+
+// Split the prefix so that (sequences x kv heads x row blocks x splits) fills about two
+// CTAs per SM; a split never spans more than 32 tiles of 64 keys.
+AttnPlan plan_attention(const eagle_shape_t* s) {
+  AttnPlan p{};
+  const int G = s->num_q_heads / s->num_kv_heads;
+  const int R = G * s->num_nodes;
+  p.row_blocks = (R + kAttnRows - 1) / kAttnRows;
+  const int max_tiles = (s->max_prefix_len + kAttnKeys - 1) / kAttnKeys;
+  const long base = static_cast<long>(s->batch) * s->num_kv_heads * p.row_blocks;
+  const long want = (2L * kNumSMs + base - 1) / base;
+  int tiles_per = static_cast<int>((max_tiles + want - 1) / want);
+  if (tiles_per < 1) tiles_per = 1;
+  if (tiles_per > 32) tiles_per = 32;
+  p.tiles_per_split = tiles_per;
+  p.splits = max_tiles > 0 ? (max_tiles + tiles_per - 1) / tiles_per : 1;
+  if (s->dtype != EAGLE_DTYPE_BF16 || p.splits == 1) {
+    p.splits = s->dtype == EAGLE_DTYPE_BF16 ? p.splits : 1;
+    p.acc_bytes = p.ml_bytes = 0;
+    return p;
+  }
+  const size_t rows = static_cast<size_t>(s->batch) * s->num_nodes * s->num_q_heads;
+  p.acc_bytes = align256(rows * p.splits * s->head_dim * sizeof(float));
+  p.ml_bytes = align256(rows * p.splits * 2 * sizeof(float));
+  return p;
+}
+
+struct LmPlan {
+  int chunks;
+  int bn;
+  int stages;
+  int tmem_cols;
+  size_t smem;
+};
+
+LmPlan plan_lm_head(const eagle_shape_t* s) {
+  LmPlan p{};
+  const long M = static_cast<long>(s->batch) * s->num_nodes;
+  p.chunks = static_cast<int>((M + 255) / 256);
+  const long per = (M + p.chunks - 1) / p.chunks;
+  p.bn = static_cast<int>(((per + 15) / 16) * 16);
+  const uint32_t stage = lm_stage_bytes(p.bn);
+  // small row counts: keep two CTAs per SM in flight; large ones: deepest ring in one CTA
+  if (stage * 4 <= 104 * 1024) {
+    p.stages = static_cast<int>((104 * 1024) / stage);
+  } else {
+    p.stages = static_cast<int>((200 * 1024) / stage);
+  }
+  if (p.stages > 8) p.stages = 8;
+  if (p.stages < 2) p.stages = 2;
+  int cols = 32;
+  while (cols < p.bn) cols <<= 1;
+  p.tmem_cols = cols;
+  p.smem = 1024 + static_cast<size_t>(p.stages) * stage + (2 * p.stages + 1) * 8 + 16;
+  return p;
+}
+
+struct AccPlan {
+  int cluster;
+  int slice;
+  size_t smem;
+};
+
+AccPlan plan_accept(const eagle_shape_t* s) {
+  AccPlan p{};
+  int cl = (s->vocab + 2047) / 2048;
+  if (cl < 1) cl = 1;
+  if (cl > kAccMaxCluster) cl = kAccMaxCluster;
+  p.cluster = cl;
+  const int per = (s->vocab + cl - 1) / cl;
+  p.slice = ((per + 3) / 4) * 4;
+  p.smem = static_cast<size_t>(2) * p.slice * sizeof(float);
+  return p;
+}
+
+constexpr size_t kAccMaxSmem = 200 * 1024;
+
+// ------------------------------------------------------------------ driver entry point
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r =
+      enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+          dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ per-device state
+
+struct DeviceState {
+  std::once_flag attrs_once;
+  bool attrs_ok = false;
+  std::mutex fork_mu;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+bool current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return false;
+  return *dev >= 0 && *dev < kMaxDevices;
+}
+
+bool ensure_attributes(int dev) {
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.attrs_once, [&] {
+    bool ok = true;
+    ok &= cudaFuncSetAttribute(lm_head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_attn_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<64>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_attn_bf16_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnSmem<128>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_accept_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kAccMaxSmem)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_accept_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kAccMaxSmem)) == cudaSuccess;
+    st.attrs_ok = ok;
+  });
+  return st.attrs_ok;
+}
+
+eagle_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? EAGLE_OK : EAGLE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ launches
+
+eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* kp, const void* vp,
+                             const int32_t* lens, const void* kt, const void* vt,
+                             const int32_t* parents, void* out, void* ws, cudaStream_t st) {
+  const int B = s->batch, N = s->num_nodes, Hq = s->num_q_heads, Hkv = s->num_kv_heads;
+  const int D = s->head_dim, Lmax = s->max_prefix_len;
+  const float scale = softmax_scale(s);
+  if (s->dtype == EAGLE_DTYPE_F32) {
+    const int rows = B * N * Hq;
+    const dim3 grid((rows + 3) / 4);
+    if (D == 64)
+      tree_attn_f32_kernel<64><<<grid, 128, 0, st>>>(
+          static_cast<const float*>(q), static_cast<const float*>(kp), static_cast<const float*>(vp), lens,
+          static_cast<const float*>(kt), static_cast<const float*>(vt), parents, static_cast<float*>(out), B,
+          N, Hq, Hkv, Lmax, scale);
+    else
+      tree_attn_f32_kernel<128><<<grid, 128, 0, st>>>(
+          static_cast<const float*>(q), static_cast<const float*>(kp), static_cast<const float*>(vp), lens,
+          static_cast<const float*>(kt), static_cast<const float*>(vt), parents, static_cast<float*>(out), B,
+          N, Hq, Hkv, Lmax, scale);
+    return launch_status();
+  }
+  const AttnPlan plan = plan_attention(s);
+  CUtensorMap tk, tv;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax),
+                              static_cast<cuuint64_t>(B) * Hkv};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Lmax) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kAttnKeys), 1};
+  if (!encode_bf16(&tk, kp, 3, dims, strides, box) || !encode_bf16(&tv, vp, 3, dims, strides, box))
+    return EAGLE_ERR_CUDA;
+  AttnParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k_tree = static_cast<const __nv_bfloat16*>(kt);
+  prm.v_tree = static_cast<const __nv_bfloat16*>(vt);
+  prm.prefix_lens = lens;
+  prm.parents = parents;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.part_acc = static_cast<float*>(ws);
+  prm.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.acc_bytes);
+  prm.B = B;
+  prm.N = N;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Lmax = Lmax;
+  prm.num_splits = plan.splits;
+  prm.tiles_per_split = plan.tiles_per_split;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const dim3 grid(plan.row_blocks, plan.splits, B * Hkv);
+  if (D == 64)
+    tree_attn_bf16_kernel<64><<<grid, kAttnThreads, AttnSmem<64>::kAlloc, st>>>(tk, tv, prm);
+  else
+    tree_attn_bf16_kernel<128><<<grid, kAttnThreads, AttnSmem<128>::kAlloc, st>>>(tk, tv, prm);
+  eagle_status_t rc = launch_status();
+  if (rc != EAGLE_OK || plan.splits == 1) return rc;
+  const int rows = B * N * Hq;
+  const dim3 cgrid((rows + 3) / 4);
+  if (D == 64)
+    tree_attn_combine_kernel<64><<<cgrid, 128, 0, st>>>(prm.part_acc, prm.part_ml, prm.out, rows, plan.splits);
+  else
+    tree_attn_combine_kernel<128><<<cgrid, 128, 0, st>>>(prm.part_acc, prm.part_ml, prm.out, rows, plan.splits);
+  return launch_status();
+}
+
+eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const void* w, float* logits,
+                           cudaStream_t st) {
+  const int M = s->batch * s->num_nodes, V = s->vocab, H = s->hidden;
+  if (s->dtype == EAGLE_DTYPE_F32) {
+    const dim3 grid((V + kLmF32TileV - 1) / kLmF32TileV, (M + kLmF32TileR - 1) / kLmF32TileR);
+    lm_head_f32_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(hidden), static_cast<const float*>(w),
+                                             logits, M, V, H);
+    return launch_status();
+  }
+  const LmPlan plan = plan_lm_head(s);
+  CUtensorMap tw, th;
+  const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
+  const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};
+  const cuuint64_t stride[1] = {static_cast<cuuint64_t>(H) * 2};
+  const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(kLmBlockV)};
+  const cuuint32_t hbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(plan.bn)};
+  if (!encode_bf16(&tw, w, 2, wd, stride, wbox) || !encode_bf16(&th, hidden, 2, hd, stride, hbox))
+    return EAGLE_ERR_CUDA;
+  LmTcParams prm{logits, M, V, H, plan.bn, plan.stages, plan.tmem_cols};
+  const dim3 grid(plan.chunks, (V + kLmBlockV - 1) / kLmBlockV);
+  lm_head_tc_kernel<<<grid, kLmThreads, plan.smem, st>>>(tw, th, prm);
+  return launch_status();
+}
+
+eagle_status_t run_accept(const eagle_shape_t* s, const float* logits, const float* draft,
+                          const int32_t* tokens, const int32_t* parents, float T, uint64_t seed,
+                          uint64_t offset, int32_t* acc, int32_t* alen, int32_t* next,
+                          cudaStream_t st) {
+  const AccPlan plan = plan_accept(s);
+  AccParams prm{};
+  prm.logits = logits;
+  prm.draft = draft;
+  prm.tokens = tokens;
+  prm.parents = parents;
+  prm.accepted_nodes = acc;
+  prm.accept_len = alen;
+  prm.next_token = next;
+  prm.N = s->num_nodes;
+  prm.V = s->vocab;
+  prm.slice = plan.slice;
+  prm.T = T;
+  prm.seed = seed;
+  prm.offset = offset;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(s->batch * plan.cluster);
+  cfg.blockDim = dim3(kAccThreads);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = plan.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (s->vocab % 4 == 0)
+    e = cudaLaunchKernelEx(&cfg, tree_accept_kernel<true>, prm);
+  else
+    e = cudaLaunchKernelEx(&cfg, tree_accept_kernel<false>, prm);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return EAGLE_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ argument checks
+
+eagle_status_t check_attention_args(const eagle_shape_t* s, const void* q, const void* kp,
+                                    const void* vp, const int32_t* lens, const void* kt,
+                                    const void* vt, const int32_t* parents, const void* out,
+                                    const void* ws, size_t ws_bytes) {
+  eagle_status_t rc = check_shape(s);
+  if (rc != EAGLE_OK) return rc;
+  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(kt) || !aligned16(vt) ||
+      !aligned16(out) || lens == nullptr || parents == nullptr)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  if (static_cast<long>(s->batch) * s->num_kv_heads > 65535) return EAGLE_ERR_UNSUPPORTED;
+  const size_t need = eagle_workspace_bytes(s);
+  if (ws_bytes < need) return EAGLE_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0))
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  return EAGLE_OK;
+}
+
+eagle_status_t check_lm_args(const eagle_shape_t* s, const void* hidden, const void* w,
+                             const float* logits) {
+  eagle_status_t rc = check_shape(s);
+  if (rc != EAGLE_OK) return rc;
+  if (!aligned16(hidden) || !aligned16(w) || !aligned16(logits)) return EAGLE_ERR_INVALID_ARGUMENT;
+  return EAGLE_OK;
+}
+
+eagle_status_t check_accept_args(const eagle_shape_t* s, const float* logits, const float* draft,
+                                 const int32_t* tokens, const int32_t* parents, float T,
+                                 const int32_t* acc, const int32_t* alen, const int32_t* next) {
+  eagle_status_t rc = check_shape(s);
+  if (rc != EAGLE_OK) return rc;
+  if (!aligned16(logits) || !aligned16(draft) || tokens == nullptr || parents == nullptr ||
+      acc == nullptr || alen == nullptr || next == nullptr)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  if (!(T >= 0.f) || !std::isfinite(T)) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (plan_accept(s).smem > kAccMaxSmem) return EAGLE_ERR_UNSUPPORTED;
+  return EAGLE_OK;
+}
+
+}  // namespace
+}  // namespace eagle
+
+using namespace eagle;
+
+extern "C" {
+
+const char* eagle_status_string(eagle_status_t status) {
+  switch (status) {
+    case EAGLE_OK: return "EAGLE_OK";
+    case EAGLE_ERR_INVALID_ARGUMENT: return "EAGLE_ERR_INVALID_ARGUMENT";
+    case EAGLE_ERR_UNSUPPORTED: return "EAGLE_ERR_UNSUPPORTED";
+    case EAGLE_ERR_WORKSPACE_TOO_SMALL: return "EAGLE_ERR_WORKSPACE_TOO_SMALL";
+    case EAGLE_ERR_CUDA: return "EAGLE_ERR_CUDA";
+  }
+  return "EAGLE_ERR_UNKNOWN";
+}
+
+size_t eagle_workspace_bytes(const eagle_shape_t* shape) {
+  if (check_shape(shape) != EAGLE_OK) return 0;
+  const AttnPlan p = plan_attention(shape);
+  return p.acc_bytes + p.ml_bytes;
+}
+
+eagle_status_t eagle_tree_attention(const eagle_shape_t* shape, const void* q, const void* k_prefix,
+                                    const void* v_prefix, const int32_t* prefix_lens,
+                                    const void* k_tree, const void* v_tree, const int32_t* parents,
+                                    void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  eagle_status_t rc = check_attention_args(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
+                                           parents, out, workspace, workspace_bytes);
+  if (rc != EAGLE_OK) return rc;
+  int dev;
+  if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
+  return run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
+                       workspace, static_cast<cudaStream_t>(stream));
+}
+
+eagle_status_t eagle_lm_head_logits(const eagle_shape_t* shape, const void* hidden, const void* w_lm,
+                                    float* logits, void* stream) {
+  eagle_status_t rc = check_lm_args(shape, hidden, w_lm, logits);
+  if (rc != EAGLE_OK) return rc;
+  int dev;
+  if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
+  return run_lm_head(shape, hidden, w_lm, logits, static_cast<cudaStream_t>(stream));
+}
+
+eagle_status_t eagle_tree_accept(const eagle_shape_t* shape, const float* logits, const float* draft_probs,
+                                 const int32_t* tokens, const int32_t* parents, float temperature,
+                                 uint64_t seed, uint64_t offset, int32_t* accepted_nodes,
+                                 int32_t* accept_len, int32_t* next_token, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  eagle_status_t rc = check_accept_args(shape, logits, draft_probs, tokens, parents, temperature,
+                                        accepted_nodes, accept_len, next_token);
+  if (rc != EAGLE_OK) return rc;
+  int dev;
+  if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
+  return run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed, offset,
+                    accepted_nodes, accept_len, next_token, static_cast<cudaStream_t>(stream));
+}
+
+eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, const void* k_prefix,
+                                 const void* v_prefix, const int32_t* prefix_lens, const void* k_tree,
+                                 const void* v_tree, const int32_t* parents, const void* hidden,
+                                 const void* w_lm, const float* draft_probs, const int32_t* tokens,
+                                 float temperature, uint64_t seed, uint64_t offset, void* out,
+                                 float* logits, int32_t* accepted_nodes, int32_t* accept_len,
+                                 int32_t* next_token, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  eagle_status_t rc = check_attention_args(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
+                                           parents, out, workspace, workspace_bytes);
+  if (rc == EAGLE_OK) rc = check_lm_args(shape, hidden, w_lm, logits);
+  if (rc == EAGLE_OK)
+    rc = check_accept_args(shape, logits, draft_probs, tokens, parents, temperature, accepted_nodes,
+                           accept_len, next_token);
+  if (rc != EAGLE_OK) return rc;
+  int dev;
+  if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DeviceState& ds = g_dev[dev];
+  std::lock_guard<std::mutex> lock(ds.fork_mu);
+  if (ds.side == nullptr) {
+    if (cudaStreamCreateWithFlags(&ds.side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ds.ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ds.ev_join, cudaEventDisableTiming) != cudaSuccess)
+      return EAGLE_ERR_CUDA;
+  }
+  // attention on the side stream (its output does not feed the walk) overlaps the
+  // LM head and the walk on the caller's stream; the caller's stream then joins it
+  if (cudaEventRecord(ds.ev_fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(ds.side, ds.ev_fork, 0) != cudaSuccess)
+    return EAGLE_ERR_CUDA;
+  rc = run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out, workspace,
+                     ds.side);
+  const eagle_status_t rc_lm = run_lm_head(shape, hidden, w_lm, logits, st);
+  const eagle_status_t rc_acc =
+      rc_lm == EAGLE_OK ? run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed,
+                                     offset, accepted_nodes, accept_len, next_token, st)
+                        : rc_lm;
+  if (cudaEventRecord(ds.ev_join, ds.side) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ds.ev_join, 0) != cudaSuccess)
+    return EAGLE_ERR_CUDA;
+  if (rc != EAGLE_OK) return rc;
+  return rc_acc;
+}
+
+eagle_status_t eagle_device_error(int32_t* code, int32_t reset) {
+  if (code == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof v) != cudaSuccess) return EAGLE_ERR_CUDA;
+  *code = v;
+  if (reset) {
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) return EAGLE_ERR_CUDA;
+  }
+  return EAGLE_OK;
+}
+
+}  // extern "C"

@@ -9,6 +9,7 @@ import ctypes
 import json
 import os
 import subprocess
+import zlib
 
 import numpy as np
 import pytest
@@ -80,7 +81,7 @@ ATTN_CASES = [
 @pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: f"B{c[0]}N{c[1]}H{c[2]}/{c[3]}D{c[4]}L{c[5]}{c[7]}")
 def test_tree_attention_matches_oracle(cuda_lib, orc, case):
     B, N, Hq, Hkv, D, Lmax, lens, dtype = case
-    rng = np.random.default_rng(hash(case) % (1 << 31))
+    rng = np.random.default_rng(zlib.crc32(repr(case).encode()))
     inp = _attn_case(rng, B, N, Hq, Hkv, D, Lmax, lens, dtype)
     got = _run_attention(cuda_lib, inp, dtype)
     ref = orc.tree_attention(**inp)
@@ -166,7 +167,8 @@ def _accept_inputs(rng, B, N, V, T, max_depth=5, dup_draft=True):
                 order = np.argsort(-logits[b, u] + rng.standard_normal(V) * 0.3)
                 picks = order[:len(ch[u])]
             else:
-                picks = rng.choice(V, size=len(ch[u]), p=row.astype(np.float64) / row.sum())
+                r64 = row.astype(np.float64)
+                picks = rng.choice(V, size=len(ch[u]), p=r64 / r64.sum())
             for c, t in zip(ch[u], picks):
                 tokens[b, c] = t
                 draft[b, c] = row

@@ -18,7 +18,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -57,58 +56,65 @@ def step_bytes(w, prefix_lens):
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event reasons through NVML every 20 ms while
+    the timed region runs (read-only queries)."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, device_index: int):
         self.idx = device_index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _sample(self, nv, h):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.samples.append((sm, int(get(h))))
+
+    def _run(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self._physical_index())
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._sample(nv, h)
+            while not self._stop.wait(0.02):
+                self._sample(nv, h)
+            self._sample(nv, h)
+        except Exception as e:  # clocks are reported as unavailable, never fatal
+            self.error = repr(e)
+
+    def _physical_index(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            ids = [v for v in vis.split(",") if v.strip()]
+            if self.idx < len(ids) and ids[self.idx].strip().isdigit():
+                return int(ids[self.idx])
+        return self.idx
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
-            self._t.start()
-        except OSError:
-            self.proc = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        time.sleep(0.05)
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        self._t.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "error": getattr(self, "error", "no samples")}
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = sorted(n for n, bit in self.REASONS.items() if mask & bit)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
 
 
 # ---------------------------------------------------------------- oracle (CPU baseline)
@@ -141,7 +147,7 @@ def oracle_step_sample(w, inp, T, lm_stride=8):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="vicuna7b_static", choices=sorted(wl.WORKLOADS))
@@ -189,6 +195,7 @@ def main():
 
     import torch
     from tree_verify_b200 import binding
+    from tree_verify_b200.replicas import max_over_ranks
     from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
 
     dist = None
@@ -216,14 +223,9 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # warm-up (also lets the clocks ramp)
     for i in range(args.warmup):
         flush.zero_()
         step.run(x, T, seed=rank, offset=i)
-    t_end = time.time() + 0.5
-    while time.time() < t_end:
-        flush.zero_()
-        step.run(x, T, seed=rank, offset=0)
     barrier()
     assert binding.device_error(reset=True) == 0
 
@@ -281,10 +283,7 @@ def main():
     assert binding.device_error(reset=True) == 0
 
     # ---- max over ranks
-    t = torch.tensor([total_ms, e2e_ms, lm_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, lm_ms = (float(v) for v in t.tolist())
+    total_ms, e2e_ms, lm_ms = max_over_ranks([total_ms, e2e_ms, lm_ms], dist, dev)
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()

@@ -163,6 +163,34 @@ eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
                                  void *stream);
 
 /*
+ * Tree attention without a caller-supplied workspace, for callers that cannot allocate
+ * device memory at call time: an inference server that plans all of its device memory at
+ * start-up and forbids allocation afterwards (cudaMalloc may synchronise the device and
+ * breaks a fixed memory plan), or a host program that hands a kernel only its input and
+ * output buffers.  The pages have no counterpart of this entry point; it is a deployment
+ * convenience.
+ *
+ * Same computation, arguments, layouts and errors as eagle_tree_attention, minus
+ * `workspace`.  The split partials live in one fixed device array of
+ * EAGLE_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the library
+ * holds until the process exits.  Shapes with eagle_workspace_bytes(shape) larger than
+ * that return EAGLE_ERR_UNSUPPORTED before anything is enqueued.  Nothing in the array
+ * needs to start at zero: every partial is written before it is read.
+ *
+ * The array is shared by every call on a device and keeps the last call's contents, so
+ * two calls whose work overlaps on the GPU (different streams, or different host threads)
+ * race on it and must be ordered by the caller.  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  This entry point allocates nothing.
+ */
+#define EAGLE_STATIC_SCRATCH_BYTES (16u << 20)
+eagle_status_t eagle_tree_attention_static(const eagle_shape_t *shape, const void *q,
+                                           const void *k_prefix, const void *v_prefix,
+                                           const int32_t *prefix_lens, const void *k_tree,
+                                           const void *v_tree, const int32_t *parents,
+                                           void *out, void *stream);
+
+/*
  * Reads (and, if `reset` != 0, clears) the device error word that bounded waits set
  * when they give up.  Synchronises the current device.  *code = 0 means no error.
  */

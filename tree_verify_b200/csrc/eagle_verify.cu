@@ -493,3 +493,51 @@ eagle_status_t eagle_device_error(int32_t* code, int32_t reset) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free variant
+// Tree attention whose split partials live in a fixed array of this library instead of a
+// caller workspace, for callers that cannot allocate device memory at call time.
+
+namespace eagle {
+namespace {
+
+static __device__ __align__(256) uint8_t g_static_scratch[EAGLE_STATIC_SCRATCH_BYTES];
+
+struct StaticScratch {
+  std::once_flag once;
+  cudaError_t status = cudaErrorUnknown;
+  void* ptr = nullptr;
+};
+StaticScratch g_scratch[kMaxDevices];
+
+// The host-side name of the array is not a device address; look the address up once per
+// device, with that device current.
+void* static_scratch_address(int dev) {
+  StaticScratch& s = g_scratch[dev];
+  std::call_once(s.once, [&] {
+    s.status = cudaGetSymbolAddress(&s.ptr, g_static_scratch);
+  });
+  return s.status == cudaSuccess ? s.ptr : nullptr;
+}
+
+}  // namespace
+}  // namespace eagle
+
+extern "C" eagle_status_t eagle_tree_attention_static(const eagle_shape_t* shape, const void* q,
+                                                      const void* k_prefix, const void* v_prefix,
+                                                      const int32_t* prefix_lens, const void* k_tree,
+                                                      const void* v_tree, const int32_t* parents,
+                                                      void* out, void* stream) {
+  if (check_shape(shape) != EAGLE_OK) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (eagle_workspace_bytes(shape) > EAGLE_STATIC_SCRATCH_BYTES) return EAGLE_ERR_UNSUPPORTED;
+  int dev;
+  if (!current_device(&dev)) return EAGLE_ERR_CUDA;
+  void* scratch = static_scratch_address(dev);
+  if (scratch == nullptr) return EAGLE_ERR_CUDA;
+  eagle_status_t rc = check_attention_args(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
+                                           parents, out, scratch, EAGLE_STATIC_SCRATCH_BYTES);
+  if (rc != EAGLE_OK) return rc;
+  if (!ensure_attributes(dev)) return EAGLE_ERR_CUDA;
+  return run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
+                       scratch, static_cast<cudaStream_t>(stream));
+}

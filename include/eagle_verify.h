@@ -145,11 +145,11 @@ eagle_status_t eagle_tree_accept(const eagle_shape_t *shape, const float *logits
                                  void *stream);
 
 /*
- * One whole verification step: tree attention, LM-head logits and the accept walk,
- * enqueued on `stream` (tree attention may run on an internal side stream that joins
- * `stream` before the call's work completes; the attention output does not feed the
- * walk).  Arguments as above; writes out, logits, accepted_nodes, accept_len and
- * next_token.
+ * One whole verification step: LM-head logits, the accept walk and tree attention,
+ * enqueued on `stream` in that order.  The walk may begin while the LM head drains and
+ * waits for it before reading the logits; tree attention, whose output the walk does not
+ * read, may run while the walk runs.  Arguments as above; writes out, logits,
+ * accepted_nodes, accept_len and next_token.
  */
 eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
                                  const void *k_prefix, const void *v_prefix,

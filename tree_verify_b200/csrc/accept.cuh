@@ -4,14 +4,23 @@
 // Speculative Sampling" and appendix B "Algorithm 1": the rule runs over the k candidates
 // of a node with an adjusted distribution after each rejection).
 //
-// One thread-block cluster walks one sequence.  The vocabulary is split into contiguous
-// slices, one per CTA, so every pass over V (row statistics, residual update, final
-// sample) runs on CL SMs at once with 128-bit loads; the residual distribution
-// r = max(0, p - p_hat) stays in the CTAs' shared memory (two buffers, so that a rejected
-// update with zero mass can keep the previous one) and the single entry r[t] that an
-// accept test needs is read from its owner through distributed shared memory.  Each
-// cluster-wide reduction combines per-CTA partials in rank order, so every CTA reaches
-// bit-identical decisions and the walk stays in lockstep without further communication.
+// One thread-block cluster walks one sequence; the vocabulary is split into contiguous
+// slices, one per CTA.  The walk is a chain of dependent decisions, so the kernel is built
+// for latency:
+//   - at each visited node the CTA's slice of the node's logits row and of the first
+//     children's draft rows come into shared memory at once by bulk async copies (one
+//     mbarrier per buffer); p_hat_c(t_c) and the accept uniforms are fetched or computed
+//     in the same round trip, and so are the race keys' random part ln(-ln u_v), so each
+//     later pass over V reads shared memory;
+//   - the root's draft rows are fetched before waiting for the LM-head grid (programmatic
+//     dependent launch), so they arrive while the logits are still being produced;
+//   - the residual r = max(0, p - p_hat) stays in the owners' shared memory (two buffers,
+//     so that a zero-mass update can keep the previous one); the scalars the next accept
+//     test needs (r[t], logits[t]) ride along with the reduction that precedes it;
+//   - every reduction (max / sum-exp, argmax, sum, race argmin) is a warp butterfly, a
+//     combine of the CTA's warps, and a push of the CTA's partial into every peer's shared
+//     memory with a remote mbarrier arrival; each CTA then combines the CL partials in rank
+//     order, so all CTAs reach bit-identical decisions without a cluster-wide barrier.
 // Only the accepted node indices, their count and the one extra token are written.
 #pragma once
 
@@ -22,9 +31,11 @@
 
 namespace eagle {
 
-constexpr int kAccThreads = 256;
+constexpr int kAccThreads = 512;
 constexpr int kAccWarps = kAccThreads / 32;
-constexpr int kAccMaxCluster = 8;
+constexpr int kAccMaxCluster = 16;
+constexpr int kAccMaxQBuf = 4;
+constexpr int kAccFixedBufs = 4;  // logits row, two residual buffers, race keys
 
 struct AccParams {
   const float* logits;       // [B,N,V]
@@ -35,163 +46,279 @@ struct AccParams {
   int32_t* accept_len;       // [B]
   int32_t* next_token;       // [B]
   int32_t N, V, slice;       // slice: vocabulary entries per CTA, multiple of 4
+  int32_t nq;                // draft-row prefetch buffers per CTA
   float T;
   uint64_t seed, offset;
 };
 
 // ---------------------------------------------------------------- reduction operators
-// Payload float4: .x/.y carry the value pair, .z/.w unused.
-struct OpMaxSum {  // (max y, sum exp(y - max))
+// Payload float4.  Every operator is commutative, so a butterfly leaves all lanes equal.
+// Components .z/.w of OpMaxSum and .y/.z/.w of OpSum are "owner fields": exactly one CTA
+// contributes a nonzero value (a scalar it alone holds in shared memory) and the others
+// contribute 0, so adding them broadcasts that scalar exactly.
+struct OpMaxSum {  // (max y, sum exp(y - max), owner fields)
+  static __device__ __forceinline__ float4 identity() { return make_float4(-INFINITY, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ float4 operator()(float4 a, float4 b) const {
     const float m = fmaxf(a.x, b.x);
-    if (m == -INFINITY) return make_float4(-INFINITY, 0.f, 0.f, 0.f);
-    return make_float4(m, a.y * expf(a.x - m) + b.y * expf(b.x - m), 0.f, 0.f);
+    const float s = m == -INFINITY ? 0.f : a.y * __expf(a.x - m) + b.y * __expf(b.x - m);
+    return make_float4(m, s, a.z + b.z, a.w + b.w);
   }
 };
 struct OpArgMax {  // (value, index bits): larger value, then lower index
+  static __device__ __forceinline__ float4 identity() {
+    return make_float4(-INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
+  }
   __device__ __forceinline__ float4 operator()(float4 a, float4 b) const {
     const int ia = __float_as_int(a.y), ib = __float_as_int(b.y);
     return (a.x > b.x || (a.x == b.x && ia < ib)) ? a : b;
   }
 };
 struct OpArgMin {  // (key, index bits): smaller key, then lower index
+  static __device__ __forceinline__ float4 identity() {
+    return make_float4(INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
+  }
   __device__ __forceinline__ float4 operator()(float4 a, float4 b) const {
     const int ia = __float_as_int(a.y), ib = __float_as_int(b.y);
     return (a.x < b.x || (a.x == b.x && ia < ib)) ? a : b;
   }
 };
-struct OpSum {
+struct OpSum {  // (sum, owner fields)
+  static __device__ __forceinline__ float4 identity() { return make_float4(0.f, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ float4 operator()(float4 a, float4 b) const {
-    return make_float4(a.x + b.x, 0.f, 0.f, 0.f);
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
   }
 };
 
 struct AccShared {
-  float4 slot[2];           // per-CTA partial exposed to the cluster (double buffered)
-  float4 warp_part[kAccWarps];
-  float4 bcast;
+  float4 wpart[kAccWarps];             // this CTA's warp partials
+  float4 cslot[2][kAccMaxCluster];     // partial of CTA r, pushed by r (double buffered)
+  uint64_t cbar[2];                    // counts the CL pushes of a round
+  uint64_t row_bar;
+  uint64_t q_bar[kAccMaxQBuf];
+  int32_t par[64];
+  int32_t tok[64];
   int32_t child_start[65];
   int32_t child_list[64];
   int32_t acc_nodes[64];
-  int32_t valid;
+  float qx[64];                        // p_hat_c(t_c) of the current node's children
+  float ux[64];                        // accept-test uniforms
 };
 
 __device__ __forceinline__ float4 shfl_xor4(float4 v, int off) {
   v.x = __shfl_xor_sync(0xffffffffu, v.x, off);
   v.y = __shfl_xor_sync(0xffffffffu, v.y, off);
+  v.z = __shfl_xor_sync(0xffffffffu, v.z, off);
+  v.w = __shfl_xor_sync(0xffffffffu, v.w, off);
   return v;
 }
 
-// Block reduction, then cluster exchange in rank order; every thread of every CTA returns
-// the same value.  Operators are commutative, so the butterfly leaves all lanes equal.
 template <class Op>
-__device__ __forceinline__ float4 cluster_reduce(AccShared& sh, float4 v, Op op, int& round,
-                                                 uint32_t CL) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ float4 warp_allreduce(float4 v, Op op) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v = op(v, shfl_xor4(v, off));
-  if (lane == 0) sh.warp_part[warp] = v;
-  __syncthreads();
+  return v;
+}
+
+struct NoOwner {
+  template <class Op>
+  __device__ __forceinline__ float4 operator()(Op) const {
+    return Op::identity();
+  }
+};
+
+// Cluster-wide reduction; every thread of every CTA returns the same bits.  `owner(op)` is
+// evaluated by warp 0 after the CTA's threads have synchronised (so it may read what they
+// wrote to shared memory) and folded into this CTA's partial.
+template <class Op, class Owner = NoOwner>
+__device__ __forceinline__ float4 cluster_reduce(AccShared& sh, float4 v, Op op, int& round,
+                                                 uint32_t CL, uint32_t cr, Owner owner = Owner()) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int buf = round & 1;
-  if (threadIdx.x == 0) {
-    float4 t = sh.warp_part[0];
-    for (int w = 1; w < kAccWarps; ++w) t = op(t, sh.warp_part[w]);
-    sh.slot[buf] = t;
-  }
-  cluster_sync_all();
-  if (warp == 0) {
-    float4 mine = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (static_cast<uint32_t>(lane) < CL) mine = dsmem_ld_f4(dsmem_map(smem_u32(&sh.slot[buf]), lane));
-    float4 t = make_float4(__shfl_sync(0xffffffffu, mine.x, 0), __shfl_sync(0xffffffffu, mine.y, 0),
-                           0.f, 0.f);
-    for (uint32_t r = 1; r < CL; ++r) {
-      const float4 o = make_float4(__shfl_sync(0xffffffffu, mine.x, r),
-                                   __shfl_sync(0xffffffffu, mine.y, r), 0.f, 0.f);
-      t = op(t, o);
-    }
-    if (lane == 0) sh.bcast = t;
-  }
+  v = warp_allreduce(v, op);
+  if (lane == 0) sh.wpart[warp] = v;
   __syncthreads();
+  if (warp == 0) {
+    float4 t = lane < kAccWarps ? sh.wpart[lane] : Op::identity();
+    t = op(warp_allreduce(t, op), owner(op));
+    if (static_cast<uint32_t>(lane) < CL) {
+      dsmem_st_f4(dsmem_map(smem_u32(&sh.cslot[buf][cr]), lane), t);
+      mbar_arrive_remote(dsmem_map(smem_u32(&sh.cbar[buf]), lane));
+    }
+  }
+  mbar_wait_cluster(smem_u32(&sh.cbar[buf]), (round >> 1) & 1, kErrAccClusterWait);
+  float4 t = static_cast<uint32_t>(lane) < CL ? sh.cslot[buf][lane] : Op::identity();
   ++round;
-  return sh.bcast;
+  return warp_allreduce(t, op);
 }
 
-template <bool kVec4>
-__device__ __forceinline__ float4 load4(const float* base, int v, int V) {
-  if (kVec4) return *reinterpret_cast<const float4*>(base + v);
-  float4 r;
-  r.x = v < V ? base[v] : 0.f;
-  r.y = v + 1 < V ? base[v + 1] : 0.f;
-  r.z = v + 2 < V ? base[v + 2] : 0.f;
-  r.w = v + 3 < V ? base[v + 3] : 0.f;
-  return r;
+// Bulk async copy of `bytes` (multiple of 16, both ends 16-byte aligned) into shared memory,
+// completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
-template <bool kVec4>
-__global__ void __launch_bounds__(kAccThreads) tree_accept_kernel(const AccParams prm) {
+// Fills buf[0 .. n) from src: one bulk copy (kBulk) or a cooperative copy.  With kBulk the
+// caller waits on `bar` before reading; without it the copy is complete after the next
+// wait_slice.
+template <bool kBulk>
+__device__ __forceinline__ void fetch_slice(float* buf, const float* src, int n, uint64_t* bar) {
+  if (kBulk) {
+    if (threadIdx.x == 0 && n > 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(smem_u32(bar), static_cast<uint32_t>(n) * 4u);
+      bulk_g2s(smem_u32(buf), src, static_cast<uint32_t>(n) * 4u, smem_u32(bar));
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += kAccThreads) buf[i] = src[i];
+  }
+}
+
+template <bool kBulk>
+__device__ __forceinline__ void wait_slice(uint64_t* bar, uint32_t& phase, int n) {
+  if (kBulk) {
+    if (n > 0) {
+      mbar_wait(smem_u32(bar), phase, kErrAccWait);
+      phase ^= 1u;
+    }
+  } else {
+    __syncthreads();
+  }
+}
+
+template <bool kBulk>
+__global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccParams prm) {
   __shared__ AccShared sh;
-  extern __shared__ float acc_rbuf[];  // [2][slice]
+  extern __shared__ __align__(16) float acc_dyn[];  // row | r0 | r1 | race keys | q[0..nq)
   const uint32_t CL = cluster_nctarank();
   const uint32_t cr = cluster_ctarank();
   const int b = blockIdx.x / CL;
-  const int N = prm.N, V = prm.V, slice = prm.slice;
+  const int N = prm.N, V = prm.V, slice = prm.slice, NQ = prm.nq;
   const int v_lo = static_cast<int>(cr) * slice;
-  const int v_hi = min(V, v_lo + slice);
+  const int n_loc = max(0, min(V, v_lo + slice) - v_lo);  // entries this CTA owns
   const float T = prm.T;
   const size_t seq = static_cast<size_t>(b) * N;
   const int tid = threadIdx.x;
+  float* rowbuf = acc_dyn;
+  float* rbuf = acc_dyn + slice;          // [2][slice]
+  float* ebuf = acc_dyn + 3 * slice;      // ln(-ln u_v) of the current node's race
+  float* qbuf = acc_dyn + 4 * slice;      // [NQ][slice]
 
+  // ---- tree set-up (inputs only; runs while the LM-head grid may still be running)
+  int ok = 1;
+  if (tid < N) {
+    const int p = prm.parents[seq + tid];
+    const int t = prm.tokens[seq + tid];
+    sh.par[tid] = p;
+    sh.tok[tid] = t;
+    ok = tid == 0 ? (p == -1) : (p >= 0 && p < tid && t >= 0 && t < V);
+  }
   if (tid == 0) {
-    const int32_t* par = prm.parents + seq;
-    const int32_t* tok = prm.tokens + seq;
-    int ok = par[0] == -1;
-    for (int i = 1; i < N; ++i) {
-      const int p = par[i];
-      if (p < 0 || p >= i) ok = 0;
-      if (tok[i] < 0 || tok[i] >= V) ok = 0;
-    }
-    sh.valid = ok;
-    if (ok) {  // children lists in ascending index (counting sort over parents)
-      for (int i = 0; i <= N; ++i) sh.child_start[i] = 0;
-      for (int i = 1; i < N; ++i) sh.child_start[par[i] + 1]++;
-      for (int i = 0; i < N; ++i) sh.child_start[i + 1] += sh.child_start[i];
-      int fill[64];
-      for (int i = 0; i < N; ++i) fill[i] = sh.child_start[i];
-      for (int i = 1; i < N; ++i) sh.child_list[fill[par[i]]++] = i;
-    }
+    mbar_init(smem_u32(&sh.cbar[0]), CL);
+    mbar_init(smem_u32(&sh.cbar[1]), CL);
+    mbar_init(smem_u32(&sh.row_bar), 1);
+    for (int q = 0; q < kAccMaxQBuf; ++q) mbar_init(smem_u32(&sh.q_bar[q]), 1);
+    fence_mbar_init();
+  }
+  ok = __syncthreads_and(ok);
+  if (ok && tid <= N) {
+    // start of node u's children list = number of drafted nodes whose parent is < u
+    int start = 0;
+    for (int i = 1; i < N; ++i) start += sh.par[i] < tid;
+    sh.child_start[tid] = start;
   }
   __syncthreads();
-  if (!sh.valid) {
+  if (ok && tid >= 1 && tid < N) {
+    // children in ascending index: earlier siblings come first
+    const int p = sh.par[tid];
+    int pos = sh.child_start[p];
+    for (int j = 1; j < tid; ++j) pos += sh.par[j] == p;
+    sh.child_list[pos] = tid;
+  }
+  // peers' barriers must be initialised before anyone pushes to them
+  cluster_sync_all();
+  if (!ok) {
+    pdl_wait();
     if (cr == 0 && tid == 0) {
       for (int i = 0; i < N; ++i) prm.accepted_nodes[seq + i] = -1;
       prm.accept_len[b] = -1;
       prm.next_token[b] = -1;
     }
-    return;  // every CTA of the cluster takes this branch; no shared memory was exchanged
+    return;  // every CTA of the cluster takes this branch; nothing was exchanged
   }
 
-  float* rbuf0 = acc_rbuf;
+  uint32_t row_phase = 0, q_phase[kAccMaxQBuf] = {0u, 0u, 0u, 0u};
   int round = 0;
   int cur = 0, nacc = 0, next = -1;
+  const float invT = T > 0.f ? 1.0f / T : 0.f;
+  // does this CTA own vocabulary entry x (and is x a real token)?
+  auto owns = [&](int x) { return x >= v_lo && x < v_lo + n_loc; };
+
+  // draft side of a node: candidate rows, p_hat_c(t_c) and the accept uniforms
+  auto issue_draft = [&](int node) {
+    const int c_begin = sh.child_start[node];
+    const int kids = sh.child_start[node + 1] - c_begin;
+    const int pre = min(kids, NQ);
+    for (int j = 0; j < pre; ++j)
+      fetch_slice<kBulk>(qbuf + j * slice, prm.draft + (seq + sh.child_list[c_begin + j]) * V + v_lo,
+                         n_loc, &sh.q_bar[j]);
+    if (tid < kids) {
+      const int c = sh.child_list[c_begin + tid];
+      sh.qx[tid] = prm.draft[(seq + c) * V + sh.tok[c]];
+      sh.ux[tid] = uniform_at(prm.seed, prm.offset, b, c, 0, 0);
+    }
+  };
+  if (T > 0.f) issue_draft(0);
+
+  // the logits come from the LM-head grid launched just before this one
+  pdl_wait();
+  // the kernel queued after this one (tree attention) does not read anything this walk
+  // writes; let it fill the SMs the walk leaves idle
+  pdl_launch_dependents();
+
   for (int depth = 0; depth < N; ++depth) {
     const float* row = prm.logits + (seq + cur) * V;
+    const int c_begin = sh.child_start[cur], c_end = sh.child_start[cur + 1];
+    const int kids = c_end - c_begin;
+    if (depth > 0 && T > 0.f) issue_draft(cur);
+    fetch_slice<kBulk>(rowbuf, row + v_lo, n_loc, &sh.row_bar);
+    if (T > 0.f) {
+      // race keys' random part for this node, while the copies are in flight
+      for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
+        const Philox4 rnd =
+            philox_group(prm.seed, prm.offset, b, cur, 1, static_cast<uint32_t>(v_lo + i) >> 2);
+        float4 e4;
+        e4.x = logf(-logf(word_to_uniform(rnd.w[0])));
+        e4.y = logf(-logf(word_to_uniform(rnd.w[1])));
+        e4.z = logf(-logf(word_to_uniform(rnd.w[2])));
+        e4.w = logf(-logf(word_to_uniform(rnd.w[3])));
+        *reinterpret_cast<float4*>(ebuf + i) = e4;
+      }
+    }
+    wait_slice<kBulk>(&sh.row_bar, row_phase, n_loc);
+    __syncthreads();  // qx / ux / race keys visible
+
     if (T == 0.f) {
       // greedy: argmax of the target logits, lowest index on ties
-      float4 best = make_float4(-INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
-      for (int v = v_lo + 4 * tid; v < v_hi; v += 4 * kAccThreads) {
-        const float4 x = load4<kVec4>(row, v, V);
+      float4 best = OpArgMax::identity();
+      for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
+        const float4 x = *reinterpret_cast<const float4*>(rowbuf + i);
         const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (v + e < v_hi && xs[e] > best.x) best = make_float4(xs[e], __int_as_float(v + e), 0.f, 0.f);
+          if (i + e < n_loc && xs[e] > best.x)
+            best = make_float4(xs[e], __int_as_float(v_lo + i + e), 0.f, 0.f);
       }
-      const float4 r = cluster_reduce(sh, best, OpArgMax(), round, CL);
+      const float4 r = cluster_reduce(sh, best, OpArgMax(), round, CL, cr);
       int m = __float_as_int(r.y);
       if (m < 0 || m >= V) m = 0;  // all-NaN row
       int match = -1;
-      for (int ci = sh.child_start[cur]; ci < sh.child_start[cur + 1]; ++ci) {
+      for (int ci = c_begin; ci < c_end; ++ci) {
         const int c = sh.child_list[ci];
-        if (prm.tokens[seq + c] == m) {
+        if (sh.tok[c] == m) {
           match = c;
           break;
         }
@@ -206,117 +333,144 @@ __global__ void __launch_bounds__(kAccThreads) tree_accept_kernel(const AccParam
       break;
     }
 
-    // p = softmax(logits[cur] / T): row statistics (M, Z) of y = l / T
-    float4 ms = make_float4(-INFINITY, 0.f, 0.f, 0.f);
-    for (int v = v_lo + 4 * tid; v < v_hi; v += 4 * kAccThreads) {
-      const float4 x = load4<kVec4>(row, v, V);
+    // p = softmax(logits[cur] / T): statistics (M, Z) of y = l / T; the owner of the first
+    // candidate's token also broadcasts its logit
+    const int x0 = kids > 0 ? sh.tok[sh.child_list[c_begin]] : -1;
+    float4 ms = OpMaxSum::identity();
+    for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
+      const float4 x = *reinterpret_cast<const float4*>(rowbuf + i);
       const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if (v + e >= v_hi) break;
-        const float y = xs[e] / T;
+        if (i + e >= n_loc) break;
+        const float y = xs[e] * invT;
         if (y > ms.x) {
-          ms.y = ms.y * expf(ms.x - y) + 1.f;
+          ms.y = ms.y * __expf(ms.x - y) + 1.f;
           ms.x = y;
         } else {
-          ms.y += expf(y - ms.x);
+          ms.y += __expf(y - ms.x);
         }
       }
     }
-    const float4 st = cluster_reduce(sh, ms, OpMaxSum(), round, CL);
-    const float M = st.x, Z = st.y;
+    const float4 st = cluster_reduce(sh, ms, OpMaxSum(), round, CL, cr, [&](OpMaxSum) {
+      float4 o = OpMaxSum::identity();
+      if (owns(x0)) o.z = rowbuf[x0 - v_lo];
+      return o;
+    });
+    const float M = st.x, invZ = 1.0f / st.y;
+    float px_next = __expf(st.z * invT - M) * invZ;  // p at the first candidate's token
 
     bool has_res = false;
     int cb = 0;
-    float Zr = 0.f;
-    int accepted = -1;
-    for (int ci = sh.child_start[cur]; ci < sh.child_start[cur + 1]; ++ci) {
-      const int c = sh.child_list[ci];
-      const int x = prm.tokens[seq + c];
-      float px;
-      if (has_res) {
-        const int owner = x / slice;
-        const uint32_t la = smem_u32(rbuf0 + cb * slice + (x - owner * slice));
-        px = dsmem_ld_f32(dsmem_map(la, owner)) / Zr;
-      } else {
-        px = expf(row[x] / T - M) / Z;
-      }
-      const float* qrow = prm.draft + (seq + c) * V;
-      const float qx = qrow[x];
-      const float u = uniform_at(prm.seed, prm.offset, b, c, 0, 0);
-      if (qx == 0.f || u < px / qx) {
-        accepted = c;
+    float invZr = 0.f;
+    int j_acc = -1;
+    for (int j = 0; j < kids; ++j) {
+      const int c = sh.child_list[c_begin + j];
+      const float px = px_next;
+      const float qx = sh.qx[j];
+      if (qx == 0.f || sh.ux[j] < px / qx) {
+        j_acc = j;
         break;
       }
       // rejected: p <- norm(max(0, p - p_hat_c)); stored unnormalised with its mass
+      const int qb = j % NQ;
+      float* q = qbuf + qb * slice;
+      if (!kBulk && j >= NQ) fetch_slice<kBulk>(q, prm.draft + (seq + c) * V + v_lo, n_loc, &sh.q_bar[qb]);
+      wait_slice<kBulk>(&sh.q_bar[qb], q_phase[qb], n_loc);
       const int nb = has_res ? (cb ^ 1) : cb;
-      float* dst = rbuf0 + nb * slice;
-      const float* src = rbuf0 + cb * slice;
+      float* dst = rbuf + nb * slice;
+      const float* src = rbuf + cb * slice;
       float part = 0.f;
-      for (int v = v_lo + 4 * tid; v < v_hi; v += 4 * kAccThreads) {
-        const float4 q4 = load4<kVec4>(qrow, v, V);
-        float pv[4];
+      for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
+        const float4 q4 = *reinterpret_cast<const float4*>(q + i);
+        float4 p4;
         if (has_res) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) pv[e] = src[v - v_lo + e] / Zr;
+          const float4 s4 = *reinterpret_cast<const float4*>(src + i);
+          p4 = make_float4(s4.x * invZr, s4.y * invZr, s4.z * invZr, s4.w * invZr);
         } else {
-          const float4 x4 = load4<kVec4>(row, v, V);
-          pv[0] = expf(x4.x / T - M) / Z;
-          pv[1] = expf(x4.y / T - M) / Z;
-          pv[2] = expf(x4.z / T - M) / Z;
-          pv[3] = expf(x4.w / T - M) / Z;
+          const float4 x4 = *reinterpret_cast<const float4*>(rowbuf + i);
+          p4 = make_float4(__expf(x4.x * invT - M) * invZ, __expf(x4.y * invT - M) * invZ,
+                           __expf(x4.z * invT - M) * invZ, __expf(x4.w * invT - M) * invZ);
         }
-        const float qs[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float r = (v + e < v_hi) ? fmaxf(pv[e] - qs[e], 0.f) : 0.f;
-          dst[v - v_lo + e] = r;
-          part += r;
-        }
+        float4 r4 = make_float4(fmaxf(p4.x - q4.x, 0.f), fmaxf(p4.y - q4.y, 0.f),
+                                fmaxf(p4.z - q4.z, 0.f), fmaxf(p4.w - q4.w, 0.f));
+        if (i + 1 >= n_loc) r4.y = 0.f;
+        if (i + 2 >= n_loc) r4.z = 0.f;
+        if (i + 3 >= n_loc) r4.w = 0.f;
+        *reinterpret_cast<float4*>(dst + i) = r4;
+        part += (r4.x + r4.y) + (r4.z + r4.w);
       }
-      const float4 tot = cluster_reduce(sh, make_float4(part, 0.f, 0.f, 0.f), OpSum(), round, CL);
+      // the owner of the next candidate's token broadcasts what its accept test may need:
+      // the new residual there, the previous one, and the logit
+      const int xn = j + 1 < kids ? sh.tok[sh.child_list[c_begin + j + 1]] : -1;
+      const float4 tot = cluster_reduce(sh, make_float4(part, 0.f, 0.f, 0.f), OpSum(), round, CL, cr,
+                                        [&](OpSum) {
+                                          float4 o = OpSum::identity();
+                                          if (owns(xn)) {
+                                            o.y = dst[xn - v_lo];
+                                            o.z = has_res ? src[xn - v_lo] : 0.f;
+                                            o.w = rowbuf[xn - v_lo];
+                                          }
+                                          return o;
+                                        });
       if (tot.x > 0.f) {
         cb = nb;
-        Zr = tot.x;
+        invZr = 1.0f / tot.x;
         has_res = true;
+        px_next = tot.y * invZr;
+      } else {
+        // zero residual mass: p is kept
+        px_next = has_res ? tot.z * invZr : __expf(tot.w * invT - M) * invZ;
       }
+      // every thread of this CTA is past its reads of buffer qb (the reduction above
+      // synchronised the CTA): refill it with a later candidate's row
+      if (kBulk && j + NQ < kids)
+        fetch_slice<kBulk>(q, prm.draft + (seq + sh.child_list[c_begin + j + NQ]) * V + v_lo, n_loc,
+                           &sh.q_bar[qb]);
     }
-    if (accepted >= 0) {
-      if (tid == 0) sh.acc_nodes[nacc] = accepted;
+    if (j_acc >= 0) {
+      const int c = sh.child_list[c_begin + j_acc];
+      if (tid == 0) sh.acc_nodes[nacc] = c;
       ++nacc;
-      cur = accepted;
+      // candidates [j_acc, j_acc + NQ) may still have draft-row copies in flight: land them
+      // before their buffers are reused
+      if (kBulk)
+        for (int j = j_acc; j < min(kids, j_acc + NQ); ++j)
+          wait_slice<kBulk>(&sh.q_bar[j % NQ], q_phase[j % NQ], n_loc);
+      __syncthreads();
+      cur = c;
       continue;
     }
 
     // no child accepted: exponential race over the current distribution,
     // key_v = ln(-ln u_v) - ln w_v with w = residual r or exp(y - M)
-    float4 best = make_float4(INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
-    const float* src = rbuf0 + cb * slice;
-    for (int v = v_lo + 4 * tid; v < v_hi; v += 4 * kAccThreads) {
-      const Philox4 rnd = philox_group(prm.seed, prm.offset, b, cur, 1, static_cast<uint32_t>(v) >> 2);
+    float4 best = OpArgMin::identity();
+    const float* src = rbuf + cb * slice;
+    for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
+      const float4 e4 = *reinterpret_cast<const float4*>(ebuf + i);
+      const float es[4] = {e4.x, e4.y, e4.z, e4.w};
       float lw[4];
       if (has_res) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float r = src[v - v_lo + e];
-          lw[e] = r > 0.f ? logf(r) : -INFINITY;
-        }
+        const float4 s4 = *reinterpret_cast<const float4*>(src + i);
+        lw[0] = s4.x > 0.f ? __logf(s4.x) : -INFINITY;
+        lw[1] = s4.y > 0.f ? __logf(s4.y) : -INFINITY;
+        lw[2] = s4.z > 0.f ? __logf(s4.z) : -INFINITY;
+        lw[3] = s4.w > 0.f ? __logf(s4.w) : -INFINITY;
       } else {
-        const float4 x4 = load4<kVec4>(row, v, V);
-        lw[0] = x4.x / T - M;
-        lw[1] = x4.y / T - M;
-        lw[2] = x4.z / T - M;
-        lw[3] = x4.w / T - M;
+        const float4 x4 = *reinterpret_cast<const float4*>(rowbuf + i);
+        lw[0] = x4.x * invT - M;
+        lw[1] = x4.y * invT - M;
+        lw[2] = x4.z * invT - M;
+        lw[3] = x4.w * invT - M;
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if (v + e >= v_hi || lw[e] == -INFINITY) continue;
-        const float u = word_to_uniform(rnd.w[e]);
-        const float key = logf(-logf(u)) - lw[e];
-        if (key < best.x) best = make_float4(key, __int_as_float(v + e), 0.f, 0.f);
+        if (i + e >= n_loc || lw[e] == -INFINITY) continue;
+        const float key = es[e] - lw[e];
+        if (key < best.x) best = make_float4(key, __int_as_float(v_lo + i + e), 0.f, 0.f);
       }
     }
-    const float4 r = cluster_reduce(sh, best, OpArgMin(), round, CL);
+    const float4 r = cluster_reduce(sh, best, OpArgMin(), round, CL, cr);
     next = __float_as_int(r.y);
     if (next < 0 || next >= V) next = 0;
     break;
@@ -327,8 +481,9 @@ __global__ void __launch_bounds__(kAccThreads) tree_accept_kernel(const AccParam
     prm.accept_len[b] = nacc;
     prm.next_token[b] = next;
   }
-  // no CTA may leave while a peer can still read its shared memory
-  cluster_sync_all();
+  // Every peer's pushes into this CTA were awaited in the last reduction, and every remote
+  // read of a residual entry precedes its reader's next push, so no peer can still touch
+  // this CTA's shared memory: no closing cluster barrier is needed.
 }
 
 }  // namespace eagle

@@ -11,13 +11,14 @@
 // block of 64 query rows, prefix split).  The query rows of a kv head are the G heads x N
 // nodes that share it (row r -> node r / G, head g*G + r % G), so every prefix K/V tile is
 // brought from HBM into shared memory once by TMA (128-byte swizzled boxes) and used by
-// all of them.  A producer warp streams 64-key K/V tiles through a two-stage mbarrier
-// ring; four consumer warps each own 16 query rows and run S = Q K^T and O += P V with
-// warp-level bf16 MMAs and an online softmax kept in registers (quad shuffles for the row
-// max).  The CTA of the last split also runs the tree tile: the N tree keys, masked by
-// the per-node ancestor bitmask anc[i] = anc[parent(i)] | 1 << i built in shared memory.
-// Splits write (m, l, acc) partials that a second kernel merges by log-sum-exp; with a
-// single split the CTA normalises and writes the output itself.
+// all of them.  A producer warp streams 64-key K/V tiles through a multi-stage mbarrier
+// ring (a split's tiles are all in flight at once); four consumer warps each own 16 query
+// rows and run S = Q K^T and O += P V with warp-level bf16 MMAs and an online softmax kept
+// in registers (quad shuffles for the row max).  The CTA of the last split also runs the
+// tree tile: the N tree keys, masked by the per-node ancestor bitmask (node i and every
+// node up its parent chain) built in shared memory.  Splits write (m, l, acc) partials
+// that a second kernel merges by log-sum-exp; with a single split the CTA normalises and
+// writes the output itself.
 //
 // f32 path: one warp per output row, fp32 SIMT, keys streamed in order (small shapes).
 #pragma once
@@ -30,7 +31,13 @@ constexpr int kAttnKeys = 64;        // keys per tile
 constexpr int kAttnRows = 64;        // query rows per CTA (4 consumer warps x 16)
 constexpr int kAttnConsumerWarps = 4;
 constexpr int kAttnThreads = 32 * (kAttnConsumerWarps + 1);
-constexpr int kAttnStages = 2;
+
+// K/V ring depth: the kernel's registers allow one CTA per SM, so the ring takes most of
+// the shared memory and a split's tiles are all in flight at once.
+template <int D>
+constexpr int attn_stages() {
+  return D == 128 ? 4 : 8;
+}
 
 struct AttnParams {
   const __nv_bfloat16* q;       // [B,N,Hq,D]
@@ -57,12 +64,14 @@ __device__ __forceinline__ uint32_t attn_swz(int row, int d) {
 
 template <int D>
 struct AttnSmem {
+  static constexpr int kStages = attn_stages<D>();
   static constexpr int kTileBytes = kAttnKeys * D * 2;  // one K or V tile
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kTreeOffset = kAttnStages * kStageBytes;
+  static constexpr int kTreeOffset = kStages * kStageBytes;
   static constexpr int kAncOffset = kTreeOffset + kStageBytes;
-  static constexpr int kBarOffset = kAncOffset + 64 * 8;
-  static constexpr int kBytes = kBarOffset + 2 * kAttnStages * 8 + 16;
+  static constexpr int kParOffset = kAncOffset + 64 * 8;
+  static constexpr int kBarOffset = kParOffset + 64 * 4;
+  static constexpr int kBytes = kBarOffset + 2 * kStages * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
@@ -93,13 +102,16 @@ struct AttnWarp {
     const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk += 2) {
+      // consecutive MMAs go to different accumulators (no back-to-back dependency)
+      uint32_t bh[8][2];
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(k_base + attn_swz(nt * 8 + rr, kk * 16 + mi * 8), b0, b1, b2, b3);
+        uint32_t b0, b1;
+        ldmatrix_x4(k_base + attn_swz(nt * 8 + rr, kk * 16 + mi * 8), b0, b1, bh[nt][0], bh[nt][1]);
         mma_bf16_16816(sc[nt], qf[kk], b0, b1);
-        mma_bf16_16816(sc[nt], qf[kk + 1], b2, b3);
       }
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) mma_bf16_16816(sc[nt], qf[kk + 1], bh[nt][0], bh[nt][1]);
     }
     // scale, mask, row max
     float mx[2] = {-INFINITY, -INFINITY};
@@ -171,9 +183,11 @@ __global__ void __launch_bounds__(kAttnThreads)
   extern __shared__ uint8_t attn_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(attn_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  constexpr int kStages = SM::kStages;
   uint64_t* anc = reinterpret_cast<uint64_t*>(smem + SM::kAncOffset);
+  int32_t* par_s = reinterpret_cast<int32_t*>(smem + SM::kParOffset);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBarOffset);
-  uint64_t* empty = full + kAttnStages;
+  uint64_t* empty = full + kStages;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -194,21 +208,13 @@ __global__ void __launch_bounds__(kAttnThreads)
   const uint32_t smem_base = smem_u32(smem);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kAttnStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), kAttnConsumerWarps);
     }
     fence_mbar_init();
-    if (last) {
-      // ancestor bitmasks; an out-of-range parent link ends the path at that node
-      const int32_t* par = prm.parents + static_cast<size_t>(b) * N;
-      anc[0] = 1ull;
-      for (int i = 1; i < N; ++i) {
-        const int p = par[i];
-        anc[i] = ((p >= 0 && p < i) ? anc[p] : 0ull) | (1ull << i);
-      }
-    }
   }
+  if (last && threadIdx.x < N) par_s[threadIdx.x] = prm.parents[static_cast<size_t>(b) * N + threadIdx.x];
   if (last && warp < kAttnConsumerWarps) {
     // tree K/V of (b, kvh) -> swizzled shared tile; rows >= N are zero
     const uint32_t kt = smem_base + SM::kTreeOffset;
@@ -230,6 +236,19 @@ __global__ void __launch_bounds__(kAttnThreads)
     }
   }
   __syncthreads();
+  if (last && threadIdx.x < N) {
+    // ancestor bitmask of node i: itself and every node up its parent chain; a parent link
+    // that does not point to an earlier node ends the chain
+    int a = threadIdx.x;
+    uint64_t m = 0;
+    for (int guard = 0; guard < 64 && a >= 0; ++guard) {
+      m |= 1ull << a;
+      const int p = par_s[a];
+      a = (p >= 0 && p < a) ? p : -1;
+    }
+    anc[threadIdx.x] = m;
+  }
+  __syncthreads();
 
   if (warp == kAttnConsumerWarps) {
     // ---------------- producer: prefix K/V tiles of this split
@@ -238,8 +257,8 @@ __global__ void __launch_bounds__(kAttnThreads)
       int issued = 0;
       bool ok = true;
       for (int t = 0; t < nt; ++t) {
-        const int s = t % kAttnStages;
-        const int n = t / kAttnStages;
+        const int s = t % kStages;
+        const int n = t / kStages;
         if (n > 0 && !mbar_wait(smem_u32(&empty[s]), (n - 1) & 1, kErrAttnProducerWait)) {
           ok = false;
           break;
@@ -257,8 +276,8 @@ __global__ void __launch_bounds__(kAttnThreads)
         issued = t + 1;
       }
       if (!ok) {
-        for (int t = (issued > kAttnStages ? issued - kAttnStages : 0); t < issued; ++t)
-          mbar_wait(smem_u32(&full[t % kAttnStages]), (t / kAttnStages) & 1, kErrAttnProducerWait);
+        for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
+          mbar_wait(smem_u32(&full[t % kStages]), (t / kStages) & 1, kErrAttnProducerWait);
       }
     }
     return;
@@ -294,8 +313,8 @@ __global__ void __launch_bounds__(kAttnThreads)
 
   bool ok = true;
   for (int t = 0; t < nt; ++t) {
-    const int s = t % kAttnStages;
-    if (!mbar_wait(smem_u32(&full[s]), (t / kAttnStages) & 1, kErrAttnConsumerWait)) {
+    const int s = t % kStages;
+    if (!mbar_wait(smem_u32(&full[s]), (t / kStages) & 1, kErrAttnConsumerWait)) {
       ok = false;
       break;
     }
@@ -361,7 +380,9 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
 }
 
-// Log-sum-exp merge of split partials: one warp per output row.
+// Log-sum-exp merge of split partials: one warp per output row.  The splits' (m, l) and
+// accumulators are loaded eight splits at a time with every load issued before any is
+// used, so a row costs about one memory round trip per eight splits.
 template <int D>
 __global__ void __launch_bounds__(128)
     tree_attn_combine_kernel(const float* __restrict__ part_acc, const float* __restrict__ part_ml,
@@ -369,29 +390,48 @@ __global__ void __launch_bounds__(128)
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
+  constexpr int kPer = D / 32;
+  constexpr int kBatch = 8;
   const float* ml = part_ml + static_cast<size_t>(row) * splits * 2;
   float mmax = -INFINITY;
-  for (int s = 0; s < splits; ++s) mmax = fmaxf(mmax, ml[2 * s]);
-  constexpr int kPer = D / 32;
+  for (int s = lane; s < splits; s += 32) mmax = fmaxf(mmax, ml[2 * s]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, off));
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
   float den = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = ml[2 * s];
-    if (ms == -INFINITY) continue;
-    const float w = exp2f(ms - mmax);
-    den += w * ml[2 * s + 1];
-    const float* src = part_acc + (static_cast<size_t>(row) * splits + s) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(src);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
-      acc[2] += w * v.z;
-      acc[3] += w * v.w;
-    } else {
+  for (int s0 = 0; s0 < splits; s0 += kBatch) {
+    float2 mls[kBatch];
+    float v[kBatch][kPer];
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+    for (int k = 0; k < kBatch; ++k) {
+      const int s = s0 + k;
+      if (s < splits) {
+        mls[k] = *reinterpret_cast<const float2*>(ml + 2 * s);
+        const float* src = part_acc + (static_cast<size_t>(row) * splits + s) * D + lane * kPer;
+        if constexpr (kPer == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(src);
+          v[k][0] = t.x;
+          v[k][1] = t.y;
+          v[k][2] = t.z;
+          v[k][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(src);
+          v[k][0] = t.x;
+          v[k][1] = t.y;
+        }
+      } else {
+        mls[k] = make_float2(-INFINITY, 0.f);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      if (s0 + k >= splits || mls[k].x == -INFINITY) continue;
+      const float w = exp2f(mls[k].x - mmax);
+      den += w * mls[k].y;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] += w * v[k][e];
     }
   }
   const float inv = 1.0f / den;

@@ -58,8 +58,9 @@ struct AttnPlan {
   size_t ml_bytes;
 };
 
-// Split the prefix so that (sequences x kv heads x row blocks x splits) fills about two
-// CTAs per SM; a split never spans more than 32 tiles of 64 keys.
+// Split the prefix so that (sequences x kv heads x row blocks x splits) fills one wave of
+// one CTA per SM (the kernel's register use allows one); a split never spans more than 32
+// tiles of 64 keys.
 AttnPlan plan_attention(const eagle_shape_t* s) {
   AttnPlan p{};
   const int G = s->num_q_heads / s->num_kv_heads;
@@ -67,7 +68,7 @@ AttnPlan plan_attention(const eagle_shape_t* s) {
   p.row_blocks = (R + kAttnRows - 1) / kAttnRows;
   const int max_tiles = (s->max_prefix_len + kAttnKeys - 1) / kAttnKeys;
   const long base = static_cast<long>(s->batch) * s->num_kv_heads * p.row_blocks;
-  const long want = (2L * kNumSMs + base - 1) / base;
+  const long want = (static_cast<long>(kNumSMs) + base - 1) / base;
   int tiles_per = static_cast<int>((max_tiles + want - 1) / want);
   if (tiles_per < 1) tiles_per = 1;
   if (tiles_per > 32) tiles_per = 32;
@@ -117,22 +118,31 @@ LmPlan plan_lm_head(const eagle_shape_t* s) {
 struct AccPlan {
   int cluster;
   int slice;
+  int nq;
   size_t smem;
 };
 
-AccPlan plan_accept(const eagle_shape_t* s) {
+constexpr size_t kAccSmemBudget = 200 * 1024;
+
+// One cluster per sequence: 16 CTAs (a non-portable size) for large vocabularies, fewer
+// for small ones; each CTA holds its slice of the logits row, two residual buffers and
+// up to four prefetched draft rows (plus the race keys of the current node).
+AccPlan plan_accept(const eagle_shape_t* s, int max_cluster = kAccMaxCluster) {
   AccPlan p{};
-  int cl = (s->vocab + 2047) / 2048;
+  int cl = s->vocab >= 16384 ? 16 : (s->vocab + 2047) / 2048;
   if (cl < 1) cl = 1;
-  if (cl > kAccMaxCluster) cl = kAccMaxCluster;
+  if (cl > max_cluster) cl = max_cluster;
   p.cluster = cl;
   const int per = (s->vocab + cl - 1) / cl;
   p.slice = ((per + 3) / 4) * 4;
-  p.smem = static_cast<size_t>(2) * p.slice * sizeof(float);
+  const size_t row = static_cast<size_t>(p.slice) * sizeof(float);
+  const long nq = static_cast<long>(kAccSmemBudget / row) - kAccFixedBufs;
+  p.nq = static_cast<int>(nq < 0 ? 0 : (nq > kAccMaxQBuf ? kAccMaxQBuf : nq));
+  p.smem = static_cast<size_t>(kAccFixedBufs + (p.nq > 0 ? p.nq : 1)) * row;
   return p;
 }
 
-constexpr size_t kAccMaxSmem = 200 * 1024;
+constexpr size_t kAccMaxSmem = kAccSmemBudget;
 
 // ------------------------------------------------------------------ driver entry point
 
@@ -166,9 +176,7 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t*
 struct DeviceState {
   std::once_flag attrs_once;
   bool attrs_ok = false;
-  std::mutex fork_mu;
-  cudaStream_t side = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  int max_cluster = 8;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -192,6 +200,28 @@ bool ensure_attributes(int dev) {
                                static_cast<int>(kAccMaxSmem)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_accept_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kAccMaxSmem)) == cudaSuccess;
+    // 16-CTA clusters if the device can co-schedule them, else the portable 8
+    st.max_cluster = 8;
+    if (cudaFuncSetAttribute(tree_accept_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(tree_accept_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess) {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(16);
+      cfg.blockDim = dim3(kAccThreads);
+      cfg.dynamicSmemBytes = kAccMaxSmem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, tree_accept_kernel<true>, &cfg) == cudaSuccess && n >= 1)
+        st.max_cluster = 16;
+    }
+    cudaGetLastError();
     st.attrs_ok = ok;
   });
   return st.attrs_ok;
@@ -203,9 +233,12 @@ eagle_status_t launch_status() {
 
 // ------------------------------------------------------------------ launches
 
+// `pdl`: launched right behind the accept walk of the same step, whose outputs it does not
+// read; it may then start while the walk is still running.
 eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* kp, const void* vp,
                              const int32_t* lens, const void* kt, const void* vt,
-                             const int32_t* parents, void* out, void* ws, cudaStream_t st) {
+                             const int32_t* parents, void* out, void* ws, cudaStream_t st,
+                             bool pdl = false) {
   const int B = s->batch, N = s->num_nodes, Hq = s->num_q_heads, Hkv = s->num_kv_heads;
   const int D = s->head_dim, Lmax = s->max_prefix_len;
   const float scale = softmax_scale(s);
@@ -250,11 +283,22 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   prm.num_splits = plan.splits;
   prm.tiles_per_split = plan.tiles_per_split;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  const dim3 grid(plan.row_blocks, plan.splits, B * Hkv);
-  if (D == 64)
-    tree_attn_bf16_kernel<64><<<grid, kAttnThreads, AttnSmem<64>::kAlloc, st>>>(tk, tv, prm);
-  else
-    tree_attn_bf16_kernel<128><<<grid, kAttnThreads, AttnSmem<128>::kAlloc, st>>>(tk, tv, prm);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(plan.row_blocks, plan.splits, B * Hkv);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = D == 64 ? AttnSmem<64>::kAlloc : AttnSmem<128>::kAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_bf16_kernel<64>, tk, tv, prm)
+                                : cudaLaunchKernelEx(&cfg, tree_attn_bf16_kernel<128>, tk, tv, prm);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return EAGLE_ERR_CUDA;
+  }
   eagle_status_t rc = launch_status();
   if (rc != EAGLE_OK || plan.splits == 1) return rc;
   const int rows = B * N * Hq;
@@ -293,8 +337,10 @@ eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const voi
 eagle_status_t run_accept(const eagle_shape_t* s, const float* logits, const float* draft,
                           const int32_t* tokens, const int32_t* parents, float T, uint64_t seed,
                           uint64_t offset, int32_t* acc, int32_t* alen, int32_t* next,
-                          cudaStream_t st) {
-  const AccPlan plan = plan_accept(s);
+                          cudaStream_t st, bool pdl = false) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const AccPlan plan = plan_accept(s, g_dev[dev].max_cluster);
   AccParams prm{};
   prm.logits = logits;
   prm.draft = draft;
@@ -306,6 +352,7 @@ eagle_status_t run_accept(const eagle_shape_t* s, const float* logits, const flo
   prm.N = s->num_nodes;
   prm.V = s->vocab;
   prm.slice = plan.slice;
+  prm.nq = plan.nq > 0 ? plan.nq : 1;
   prm.T = T;
   prm.seed = seed;
   prm.offset = offset;
@@ -314,13 +361,17 @@ eagle_status_t run_accept(const eagle_shape_t* s, const float* logits, const flo
   cfg.blockDim = dim3(kAccThreads);
   cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = plan.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // with `pdl` (right behind the LM head of the same step): may start while the LM head
+  // drains; the kernel waits for that grid before it reads the logits
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   cudaError_t e;
   if (s->vocab % 4 == 0)
     e = cudaLaunchKernelEx(&cfg, tree_accept_kernel<true>, prm);
@@ -369,8 +420,17 @@ eagle_status_t check_accept_args(const eagle_shape_t* s, const float* logits, co
       acc == nullptr || alen == nullptr || next == nullptr)
     return EAGLE_ERR_INVALID_ARGUMENT;
   if (!(T >= 0.f) || !std::isfinite(T)) return EAGLE_ERR_INVALID_ARGUMENT;
-  if (plan_accept(s).smem > kAccMaxSmem) return EAGLE_ERR_UNSUPPORTED;
+  // host-only bound: the largest cluster any device offers; device_accept_supported()
+  // checks the current device before anything is enqueued
+  const AccPlan ap = plan_accept(s, kAccMaxCluster);
+  if (ap.nq < 1 || ap.smem > kAccMaxSmem) return EAGLE_ERR_UNSUPPORTED;
   return EAGLE_OK;
+}
+
+// The accept plan on the current device (its largest co-schedulable cluster).
+bool device_accept_supported(const eagle_shape_t* s, int dev) {
+  const AccPlan ap = plan_accept(s, g_dev[dev].max_cluster);
+  return ap.nq >= 1 && ap.smem <= kAccMaxSmem;
 }
 
 }  // namespace
@@ -431,6 +491,7 @@ eagle_status_t eagle_tree_accept(const eagle_shape_t* shape, const float* logits
   if (rc != EAGLE_OK) return rc;
   int dev;
   if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
+  if (!device_accept_supported(shape, dev)) return EAGLE_ERR_UNSUPPORTED;
   return run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed, offset,
                     accepted_nodes, accept_len, next_token, static_cast<cudaStream_t>(stream));
 }
@@ -452,32 +513,19 @@ eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, cons
   if (rc != EAGLE_OK) return rc;
   int dev;
   if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
+  if (!device_accept_supported(shape, dev)) return EAGLE_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  DeviceState& ds = g_dev[dev];
-  std::lock_guard<std::mutex> lock(ds.fork_mu);
-  if (ds.side == nullptr) {
-    if (cudaStreamCreateWithFlags(&ds.side, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ds.ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ds.ev_join, cudaEventDisableTiming) != cudaSuccess)
-      return EAGLE_ERR_CUDA;
-  }
-  // attention on the side stream (its output does not feed the walk) overlaps the
-  // LM head and the walk on the caller's stream; the caller's stream then joins it
-  if (cudaEventRecord(ds.ev_fork, st) != cudaSuccess ||
-      cudaStreamWaitEvent(ds.side, ds.ev_fork, 0) != cudaSuccess)
-    return EAGLE_ERR_CUDA;
-  rc = run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out, workspace,
-                     ds.side);
-  const eagle_status_t rc_lm = run_lm_head(shape, hidden, w_lm, logits, st);
-  const eagle_status_t rc_acc =
-      rc_lm == EAGLE_OK ? run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed,
-                                     offset, accepted_nodes, accept_len, next_token, st)
-                        : rc_lm;
-  if (cudaEventRecord(ds.ev_join, ds.side) != cudaSuccess ||
-      cudaStreamWaitEvent(st, ds.ev_join, 0) != cudaSuccess)
-    return EAGLE_ERR_CUDA;
+  // One stream, three overlapping phases: the LM head streams W over the whole GPU; the
+  // accept walk (programmatic dependent launch) sets up while the LM head drains and walks
+  // on one cluster per sequence; tree attention (its output does not feed the walk) is
+  // released by the walk and fills the SMs the walk leaves idle.
+  rc = run_lm_head(shape, hidden, w_lm, logits, st);
   if (rc != EAGLE_OK) return rc;
-  return rc_acc;
+  rc = run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed, offset,
+                  accepted_nodes, accept_len, next_token, st, /*pdl=*/true);
+  if (rc != EAGLE_OK) return rc;
+  return run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
+                       workspace, st, /*pdl=*/true);
 }
 
 eagle_status_t eagle_device_error(int32_t* code, int32_t reset) {

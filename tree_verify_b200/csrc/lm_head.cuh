@@ -80,9 +80,15 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // the walk that consumes these logits may start its prologue now; it waits for this
+  // grid's completion before reading them
+  pdl_launch_dependents();
+
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
     const uint32_t bytes = lm_stage_bytes(bn);
+    const uint64_t pol_w = l2_policy_evict_first();  // W streams through once
+    const uint64_t pol_h = l2_policy_evict_last();   // every vocabulary tile re-reads hidden
     int issued = 0;
     for (int kb = 0; kb < KB; ++kb) {
       const int s = kb % S;
@@ -94,8 +100,10 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       if (*abort_flag) break;
       const uint32_t fb = smem_u32(&full[s]);
       mbar_arrive_expect_tx(fb, bytes);
-      tma_load_2d(smem_u32(a_tiles + s * kLmBlockV * kLmBlockK * 2), &tm_w, fb, kb * kLmBlockK, v0);
-      tma_load_2d(smem_u32(b_tiles + s * bn * kLmBlockK * 2), &tm_h, fb, kb * kLmBlockK, r0);
+      tma_load_2d_hint(smem_u32(a_tiles + s * kLmBlockV * kLmBlockK * 2), &tm_w, fb, kb * kLmBlockK,
+                       v0, pol_w);
+      tma_load_2d_hint(smem_u32(b_tiles + s * bn * kLmBlockK * 2), &tm_h, fb, kb * kLmBlockK, r0,
+                       pol_h);
       issued = kb + 1;
     }
     if (*abort_flag) {

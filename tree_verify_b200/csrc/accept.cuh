@@ -10,8 +10,8 @@
 //   - at each visited node the CTA's slice of the node's logits row and of the first
 //     children's draft rows come into shared memory at once by bulk async copies (one
 //     mbarrier per buffer); p_hat_c(t_c) and the accept uniforms are fetched or computed
-//     in the same round trip, and so are the race keys' random part ln(-ln u_v), so each
-//     later pass over V reads shared memory;
+//     in the same round trip, so each later pass over V reads shared memory; the root's
+//     race keys (ln(-ln u_v)) are computed before the logits are awaited;
 //   - the root's draft rows are fetched before waiting for the LM-head grid (programmatic
 //     dependent launch), so they arrive while the logits are still being produced;
 //   - the residual r = max(0, p - p_hat) stays in the owners' shared memory (two buffers,
@@ -104,18 +104,16 @@ struct AccShared {
   float ux[64];                        // accept-test uniforms
 };
 
-__device__ __forceinline__ float4 shfl_xor4(float4 v, int off) {
-  v.x = __shfl_xor_sync(0xffffffffu, v.x, off);
-  v.y = __shfl_xor_sync(0xffffffffu, v.y, off);
-  v.z = __shfl_xor_sync(0xffffffffu, v.z, off);
-  v.w = __shfl_xor_sync(0xffffffffu, v.w, off);
-  return v;
-}
-
-template <class Op>
-__device__ __forceinline__ float4 warp_allreduce(float4 v, Op op) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v = op(v, shfl_xor4(v, off));
+// Butterfly over lanes `offs..1` that moves only the first NC components (the ones the
+// operator actually reduces); the other components stay this lane's own.
+template <int NC, class Op>
+__device__ __forceinline__ float4 warp_reduce_nc(float4 v, Op op, int offs) {
+  for (int off = offs; off > 0; off >>= 1) {
+    float4 o = Op::identity();
+    o.x = __shfl_xor_sync(0xffffffffu, v.x, off);
+    if (NC > 1) o.y = __shfl_xor_sync(0xffffffffu, v.y, off);
+    v = op(v, o);
+  }
   return v;
 }
 
@@ -125,30 +123,52 @@ struct NoOwner {
     return Op::identity();
   }
 };
+struct NoWork {
+  __device__ __forceinline__ void operator()() const {}
+};
 
-// Cluster-wide reduction; every thread of every CTA returns the same bits.  `owner(op)` is
-// evaluated by warp 0 after the CTA's threads have synchronised (so it may read what they
-// wrote to shared memory) and folded into this CTA's partial.
-template <class Op, class Owner = NoOwner>
+// Cluster-wide reduction; every thread of every CTA returns the same bits.  NC components
+// are reduced over all threads; `owner(op)` is evaluated by warp 0 after the CTA's threads
+// have synchronised (so it may read what they wrote to shared memory) and folded into this
+// CTA's partial.  Each CTA pushes its partial into every peer's slot and arrives on the
+// peer's barrier; `work()` runs while the peers' partials are on their way; then each
+// warp folds the CL slots with a butterfly.
+template <int NC, class Op, class Owner = NoOwner, class Work = NoWork>
 __device__ __forceinline__ float4 cluster_reduce(AccShared& sh, float4 v, Op op, int& round,
-                                                 uint32_t CL, uint32_t cr, Owner owner = Owner()) {
+                                                 uint32_t CL, uint32_t cr, Owner owner = Owner(),
+                                                 Work work = Work()) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int buf = round & 1;
-  v = warp_allreduce(v, op);
+  v = warp_reduce_nc<NC>(v, op, 16);
   if (lane == 0) sh.wpart[warp] = v;
   __syncthreads();
   if (warp == 0) {
     float4 t = lane < kAccWarps ? sh.wpart[lane] : Op::identity();
-    t = op(warp_allreduce(t, op), owner(op));
+    t = op(warp_reduce_nc<NC>(t, op, kAccWarps / 2), owner(op));
     if (static_cast<uint32_t>(lane) < CL) {
       dsmem_st_f4(dsmem_map(smem_u32(&sh.cslot[buf][cr]), lane), t);
       mbar_arrive_remote(dsmem_map(smem_u32(&sh.cbar[buf]), lane));
     }
   }
+  work();
   mbar_wait_cluster(smem_u32(&sh.cbar[buf]), (round >> 1) & 1, kErrAccClusterWait);
-  float4 t = static_cast<uint32_t>(lane) < CL ? sh.cslot[buf][lane] : Op::identity();
+  // lane r folds CTA r's partial; a butterfly over all 32 lanes (all four components: the
+  // owner fields ride along) leaves the same bits in every lane of every warp.  Every
+  // thread must get the result: the walk's control flow is decided from it, and a thread
+  // that decided differently would desynchronise the CTA's barriers.
+  float4 t = static_cast<uint32_t>(lane) < CL ? sh.cslot[buf][lane & (kAccMaxCluster - 1)]
+                                              : Op::identity();
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    float4 o;
+    o.x = __shfl_xor_sync(0xffffffffu, t.x, off);
+    o.y = __shfl_xor_sync(0xffffffffu, t.y, off);
+    o.z = __shfl_xor_sync(0xffffffffu, t.z, off);
+    o.w = __shfl_xor_sync(0xffffffffu, t.w, off);
+    t = op(t, o);
+  }
   ++round;
-  return warp_allreduce(t, op);
+  return t;
 }
 
 // Bulk async copy of `bytes` (multiple of 16, both ends 16-byte aligned) into shared memory,
@@ -189,6 +209,13 @@ __device__ __forceinline__ void wait_slice(uint64_t* bar, uint32_t& phase, int n
   }
 }
 
+// ln(-ln u_v) for tokens v .. v+3 of the race at `node` (v a multiple of 4).
+__device__ __forceinline__ float4 race_keys(uint64_t seed, uint64_t offset, int b, int node, int v) {
+  const Philox4 rnd = philox_group(seed, offset, b, node, 1, static_cast<uint32_t>(v) >> 2);
+  return make_float4(logf(-logf(word_to_uniform(rnd.w[0]))), logf(-logf(word_to_uniform(rnd.w[1]))),
+                     logf(-logf(word_to_uniform(rnd.w[2]))), logf(-logf(word_to_uniform(rnd.w[3]))));
+}
+
 template <bool kBulk>
 __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccParams prm) {
   __shared__ AccShared sh;
@@ -204,7 +231,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
   const int tid = threadIdx.x;
   float* rowbuf = acc_dyn;
   float* rbuf = acc_dyn + slice;          // [2][slice]
-  float* ebuf = acc_dyn + 3 * slice;      // ln(-ln u_v) of the current node's race
+  float* ebuf = acc_dyn + 3 * slice;      // ln(-ln u_v) of the root's race
   float* qbuf = acc_dyn + 4 * slice;      // [NQ][slice]
 
   // ---- tree set-up (inputs only; runs while the LM-head grid may still be running)
@@ -271,7 +298,13 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       sh.ux[tid] = uniform_at(prm.seed, prm.offset, b, c, 0, 0);
     }
   };
-  if (T > 0.f) issue_draft(0);
+  if (T > 0.f) {
+    issue_draft(0);
+    // the root's race keys (the walk most often ends there); each thread keeps the keys of
+    // the entries it later races over
+    for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads)
+      *reinterpret_cast<float4*>(ebuf + i) = race_keys(prm.seed, prm.offset, b, 0, v_lo + i);
+  }
 
   // the logits come from the LM-head grid launched just before this one
   pdl_wait();
@@ -285,21 +318,8 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     const int kids = c_end - c_begin;
     if (depth > 0 && T > 0.f) issue_draft(cur);
     fetch_slice<kBulk>(rowbuf, row + v_lo, n_loc, &sh.row_bar);
-    if (T > 0.f) {
-      // race keys' random part for this node, while the copies are in flight
-      for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
-        const Philox4 rnd =
-            philox_group(prm.seed, prm.offset, b, cur, 1, static_cast<uint32_t>(v_lo + i) >> 2);
-        float4 e4;
-        e4.x = logf(-logf(word_to_uniform(rnd.w[0])));
-        e4.y = logf(-logf(word_to_uniform(rnd.w[1])));
-        e4.z = logf(-logf(word_to_uniform(rnd.w[2])));
-        e4.w = logf(-logf(word_to_uniform(rnd.w[3])));
-        *reinterpret_cast<float4*>(ebuf + i) = e4;
-      }
-    }
     wait_slice<kBulk>(&sh.row_bar, row_phase, n_loc);
-    __syncthreads();  // qx / ux / race keys visible
+    __syncthreads();  // qx / ux visible
 
     if (T == 0.f) {
       // greedy: argmax of the target logits, lowest index on ties
@@ -312,7 +332,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
           if (i + e < n_loc && xs[e] > best.x)
             best = make_float4(xs[e], __int_as_float(v_lo + i + e), 0.f, 0.f);
       }
-      const float4 r = cluster_reduce(sh, best, OpArgMax(), round, CL, cr);
+      const float4 r = cluster_reduce<2>(sh, best, OpArgMax(), round, CL, cr);
       int m = __float_as_int(r.y);
       if (m < 0 || m >= V) m = 0;  // all-NaN row
       int match = -1;
@@ -352,11 +372,14 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
         }
       }
     }
-    const float4 st = cluster_reduce(sh, ms, OpMaxSum(), round, CL, cr, [&](OpMaxSum) {
-      float4 o = OpMaxSum::identity();
-      if (owns(x0)) o.z = rowbuf[x0 - v_lo];
-      return o;
-    });
+    const float4 st = cluster_reduce<2>(
+        sh, ms, OpMaxSum(), round, CL, cr,
+        [&](OpMaxSum) {
+          float4 o = OpMaxSum::identity();
+          if (owns(x0)) o.z = rowbuf[x0 - v_lo];
+          return o;
+        },
+        NoWork());
     const float M = st.x, invZ = 1.0f / st.y;
     float px_next = __expf(st.z * invT - M) * invZ;  // p at the first candidate's token
 
@@ -403,7 +426,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       // the owner of the next candidate's token broadcasts what its accept test may need:
       // the new residual there, the previous one, and the logit
       const int xn = j + 1 < kids ? sh.tok[sh.child_list[c_begin + j + 1]] : -1;
-      const float4 tot = cluster_reduce(sh, make_float4(part, 0.f, 0.f, 0.f), OpSum(), round, CL, cr,
+      const float4 tot = cluster_reduce<1>(sh, make_float4(part, 0.f, 0.f, 0.f), OpSum(), round, CL, cr,
                                         [&](OpSum) {
                                           float4 o = OpSum::identity();
                                           if (owns(xn)) {
@@ -447,7 +470,8 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     float4 best = OpArgMin::identity();
     const float* src = rbuf + cb * slice;
     for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
-      const float4 e4 = *reinterpret_cast<const float4*>(ebuf + i);
+      const float4 e4 = cur == 0 ? *reinterpret_cast<const float4*>(ebuf + i)
+                                 : race_keys(prm.seed, prm.offset, b, cur, v_lo + i);
       const float es[4] = {e4.x, e4.y, e4.z, e4.w};
       float lw[4];
       if (has_res) {
@@ -470,7 +494,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
         if (key < best.x) best = make_float4(key, __int_as_float(v_lo + i + e), 0.f, 0.f);
       }
     }
-    const float4 r = cluster_reduce(sh, best, OpArgMin(), round, CL, cr);
+    const float4 r = cluster_reduce<2>(sh, best, OpArgMin(), round, CL, cr);
     next = __float_as_int(r.y);
     if (next < 0 || next >= V) next = 0;
     break;

@@ -14,6 +14,7 @@
 #include "../../include/eagle_verify.h"
 #include "accept.cuh"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "device_common.cuh"
 #include "lm_head.cuh"
 
@@ -51,6 +52,7 @@ float softmax_scale(const eagle_shape_t* s) {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct AttnPlan {
+  int nodes_per_block;
   int row_blocks;
   int splits;
   int tiles_per_split;
@@ -64,8 +66,14 @@ struct AttnPlan {
 AttnPlan plan_attention(const eagle_shape_t* s) {
   AttnPlan p{};
   const int G = s->num_q_heads / s->num_kv_heads;
-  const int R = G * s->num_nodes;
-  p.row_blocks = (R + kAttnRows - 1) / kAttnRows;
+  if (s->dtype == EAGLE_DTYPE_BF16) {
+    // tensor-core path: a 128-row tile holds floor(128 / G) nodes x G heads
+    p.nodes_per_block = G <= kTcRows ? kTcRows / G : 1;
+    p.row_blocks = (s->num_nodes + p.nodes_per_block - 1) / p.nodes_per_block;
+  } else {
+    p.nodes_per_block = 0;
+    p.row_blocks = 1;
+  }
   const int max_tiles = (s->max_prefix_len + kAttnKeys - 1) / kAttnKeys;
   const long base = static_cast<long>(s->batch) * s->num_kv_heads * p.row_blocks;
   const long want = (static_cast<long>(kNumSMs) + base - 1) / base;
@@ -191,11 +199,10 @@ bool ensure_attributes(int dev) {
     bool ok = true;
     ok &= cudaFuncSetAttribute(lm_head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tree_attn_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               AttnSmem<64>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tree_attn_bf16_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               AttnSmem<128>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               TcSmem<64>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               TcSmem<128>::kAlloc) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_accept_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kAccMaxSmem)) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_accept_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -258,14 +265,23 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
     return launch_status();
   }
   const AttnPlan plan = plan_attention(s);
-  CUtensorMap tk, tv;
+  const int G = Hq / Hkv;
+  CUtensorMap tq, tk, tv;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax),
                               static_cast<cuuint64_t>(B) * Hkv};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Lmax) * D * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kAttnKeys), 1};
-  if (!encode_bf16(&tk, kp, 3, dims, strides, box) || !encode_bf16(&tv, vp, 3, dims, strides, box))
+  // queries viewed as [B*N, Hq, D]: one box = G heads x nodes_per_block nodes of a kv head
+  const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hq),
+                               static_cast<cuuint64_t>(B) * s->num_nodes};
+  const cuuint64_t qstrides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hq) * D * 2};
+  const cuuint32_t qbox[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(plan.nodes_per_block)};
+  if (!encode_bf16(&tk, kp, 3, dims, strides, box) || !encode_bf16(&tv, vp, 3, dims, strides, box) ||
+      !encode_bf16(&tq, q, 3, qdims, qstrides, qbox))
     return EAGLE_ERR_CUDA;
-  AttnParams prm{};
+  TcAttnParams tp{};
+  AttnParams& prm = tp.a;
+  tp.nodes_per_block = plan.nodes_per_block;
   prm.q = static_cast<const __nv_bfloat16*>(q);
   prm.k_tree = static_cast<const __nv_bfloat16*>(kt);
   prm.v_tree = static_cast<const __nv_bfloat16*>(vt);
@@ -275,26 +291,26 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   prm.part_acc = static_cast<float*>(ws);
   prm.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.acc_bytes);
   prm.B = B;
-  prm.N = N;
+  prm.N = s->num_nodes;
   prm.Hq = Hq;
   prm.Hkv = Hkv;
-  prm.G = Hq / Hkv;
+  prm.G = G;
   prm.Lmax = Lmax;
   prm.num_splits = plan.splits;
   prm.tiles_per_split = plan.tiles_per_split;
   prm.scale_log2 = scale * 1.4426950408889634f;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(plan.row_blocks, plan.splits, B * Hkv);
-  cfg.blockDim = dim3(kAttnThreads);
-  cfg.dynamicSmemBytes = D == 64 ? AttnSmem<64>::kAlloc : AttnSmem<128>::kAlloc;
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = D == 64 ? TcSmem<64>::kAlloc : TcSmem<128>::kAlloc;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  const cudaError_t e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_bf16_kernel<64>, tk, tv, prm)
-                                : cudaLaunchKernelEx(&cfg, tree_attn_bf16_kernel<128>, tk, tv, prm);
+  const cudaError_t e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, tq, tk, tv, tp)
+                                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, tq, tk, tv, tp);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EAGLE_ERR_CUDA;
@@ -396,6 +412,7 @@ eagle_status_t check_attention_args(const eagle_shape_t* s, const void* q, const
       !aligned16(out) || lens == nullptr || parents == nullptr)
     return EAGLE_ERR_INVALID_ARGUMENT;
   if (static_cast<long>(s->batch) * s->num_kv_heads > 65535) return EAGLE_ERR_UNSUPPORTED;
+  if (s->dtype == EAGLE_DTYPE_BF16 && s->num_q_heads / s->num_kv_heads > kTcRows) return EAGLE_ERR_UNSUPPORTED;
   const size_t need = eagle_workspace_bytes(s);
   if (ws_bytes < need) return EAGLE_ERR_WORKSPACE_TOO_SMALL;
   if (need > 0 && (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0))

@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     float* out = prm.logits;
     for (int c0 = 0; c0 < bn; c0 += 16) {
       uint32_t r[16];
+      __syncwarp();  // the TMEM load below is warp-wide
       tmem_ld_32x32b_x16(lane_base + c0, r);
       tmem_ld_wait();
       if (v < prm.V) {

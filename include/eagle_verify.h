@@ -69,7 +69,8 @@ typedef struct {
 const char *eagle_status_string(eagle_status_t status);
 
 /* Bytes of `workspace` the entry points below need for this shape (0 if the shape is
- * invalid).  The split-KV partials of tree attention live there. */
+ * invalid).  The split-KV partials of tree attention live there; for shapes that
+ * eagle_verify_step may run beside the LM head this is the larger of the two split plans. */
 size_t eagle_workspace_bytes(const eagle_shape_t *shape);
 
 /*
@@ -150,6 +151,13 @@ eagle_status_t eagle_tree_accept(const eagle_shape_t *shape, const float *logits
  * waits for it before reading the logits; tree attention, whose output the walk does not
  * read, may run while the walk runs.  Arguments as above; writes out, logits,
  * accepted_nodes, accept_len and next_token.
+ *
+ * Greedy steps (temperature 0) on bf16 shapes with few tree rows (B*N <= 48 at D = 128)
+ * instead run tree attention beside the LM head: the library enqueues it on a second
+ * stream of its own (one per device, created with two events on the first such call) that
+ * starts once the LM head's CTAs hold their SMs, and `stream` waits for it before any work
+ * enqueued after this call.  Such calls on one device are serialised on the host while
+ * they are enqueued.  The workspace from eagle_workspace_bytes() covers both schedules.
  */
 eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
                                  const void *k_prefix, const void *v_prefix,
@@ -173,8 +181,9 @@ eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
  * Same computation, arguments, layouts and errors as eagle_tree_attention, minus
  * `workspace`.  The split partials live in one fixed device array of
  * EAGLE_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads the library
- * holds until the process exits.  Shapes with eagle_workspace_bytes(shape) larger than
- * that return EAGLE_ERR_UNSUPPORTED before anything is enqueued.  Nothing in the array
+ * holds until the process exits.  Shapes whose partials for eagle_tree_attention's own
+ * split plan need more than that (for most shapes, eagle_workspace_bytes(shape)) return
+ * EAGLE_ERR_UNSUPPORTED before anything is enqueued.  Nothing in the array
  * needs to start at zero: every partial is written before it is read.
  *
  * The array is shared by every call on a device and keeps the last call's contents, so

@@ -61,8 +61,61 @@ def test_verify_step_full_size(cuda_lib, orc, name, T):
     assert exact >= B - max(1, B // 8), f"only {exact}/{B} sequences compared exactly"
 
 
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+OVERLAP_CASES = {
+    # one sequence, the bench workload's tree (45 nodes) on a shorter prefix
+    "vicuna": ("vicuna7b_static", dict(prefix_len=700, vocab=5000, hidden=1024)),
+    # two sequences of ragged length, a random tree of 20 nodes
+    "ragged": ("batched7b", dict(batch=2, tree_arg=(20, 6), prefix_len=900, prefix_min=1, vocab=5000,
+                                 hidden=1024)),
+    # head dim 64, four query heads per kv head
+    "d64": ("batched7b", dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=64, tree_arg=(20, 6),
+                              prefix_len=500, prefix_min=40, vocab=3000, hidden=512)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(OVERLAP_CASES))
+def test_verify_step_overlapped_schedule(cuda_lib, orc, case):
+    """Shapes small enough for eagle_verify_step's two-stream schedule (greedy steps:
+    attention in one-tile-per-CTA splits beside the LM head): logits and the walk are
+    bit-identical to the stage calls; the attention, merged from other splits, matches the
+    oracle and the standalone call within the bf16 tolerance."""
+    from tree_verify_b200 import binding
+    from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
+    base, kw = OVERLAP_CASES[case]
+    w = wl.scaled(wl.WORKLOADS[base], **kw)
+    inp = wl.generate(w, 1.0)
+    shape = shape_from_workload(w)
+    # the workspace is sized for the one-tile-per-CTA plan: the schedule is the overlapped one
+    rows = w.batch * w.num_nodes * w.num_q_heads
+    splits = (w.prefix_len + 63) // 64 + 1
+    assert binding.workspace_bytes(shape) == (_align256(rows * splits * w.head_dim * 4)
+                                              + _align256(rows * splits * 2 * 4))
+    x = StepInputs.from_numpy(inp, w.dtype)
+    a, b = VerifyStep(shape), VerifyStep(shape)
+    a.run(x, 0.0, 3, 4)  # the schedule that overlaps attention with the LM head is greedy-only
+    b.attention(x)
+    b.lm_head(x)
+    b.accept(x, 0.0, 3, 4)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error(reset=True) == 0
+    for name in ("logits", "accepted_nodes", "accept_len", "next_token"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    ref = orc.tree_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["prefix_lens"],
+                             inp["k_tree"], inp["v_tree"], inp["parents"])
+    got = a.out.float().cpu().numpy().reshape(-1, w.head_dim)
+    err = row_rel_err(got, ref.reshape(-1, w.head_dim))
+    assert err.max() <= TOL[w.dtype], f"attention max row error {err.max():.3e}"
+    alone = b.out.float().cpu().numpy().reshape(-1, w.head_dim)
+    assert row_rel_err(got, alone).max() <= TOL[w.dtype]
+
+
 def test_verify_step_stages_equal_fused_call(cuda_lib):
-    """The three stage entry points in sequence give the same bits as eagle_verify_step."""
+    """The three stage entry points in sequence give the same bits as eagle_verify_step
+    (a shape with too many tree rows for the overlapped schedule)."""
     from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
     w = wl.scaled(wl.WORKLOADS["batched7b"], batch=3, prefix_len=700, prefix_min=100, vocab=5000,
                   hidden=1024)
@@ -74,5 +127,6 @@ def test_verify_step_stages_equal_fused_call(cuda_lib):
     b.lm_head(x)
     b.accept(x, 1.0, 11, 12)
     torch.cuda.synchronize()
+    assert cuda_lib.device_error(reset=True) == 0
     for name in ("out", "logits", "accepted_nodes", "accept_len", "next_token"):
         assert torch.equal(getattr(a, name), getattr(b, name)), name

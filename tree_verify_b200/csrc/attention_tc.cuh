@@ -38,17 +38,21 @@ constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
 constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 2);
 constexpr float kTcRescaleThreshold = 8.0f;  // log2 units
 
-template <int D>
+// Lite: the compact layout for a CTA that runs exactly one tile (one prefix tile, or the
+// tree tile in a CTA of its own): one K/V stage, which the tree tile shares, and one P
+// buffer.  It is small enough to share an SM with two LM-head CTAs.
+template <int D, bool Lite = false>
 struct TcSmem {
-  static constexpr int kStages = D == 128 ? 3 : 6;
+  static constexpr int kStages = Lite ? 1 : (D == 128 ? 3 : 6);
+  static constexpr int kPBufs = Lite ? 1 : 2;
   static constexpr int kTile = kAttnKeys * D * 2;  // one K or V tile (D/64 boxes of 64 x 128 B)
   static constexpr int kQ = kTcRows * D * 2;        // D/64 boxes of 128 rows x 128 B
   static constexpr int kP = kTcRows * kAttnKeys * 2;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kQOff + kQ;
-  static constexpr int kTreeOff = kKVOff + kStages * 2 * kTile;
-  static constexpr int kPOff = kTreeOff + 2 * kTile;
-  static constexpr int kAncOff = kPOff + 2 * kP;
+  static constexpr int kTreeOff = Lite ? kKVOff : kKVOff + kStages * 2 * kTile;
+  static constexpr int kPOff = kKVOff + kStages * 2 * kTile + (Lite ? 0 : 2 * kTile);
+  static constexpr int kAncOff = kPOff + kPBufs * kP;
   static constexpr int kParOff = kAncOff + 64 * 8;
   // row-maximum exchange [tile parity][half][row] and, after the loop, the denominator
   // exchange [2][half][row]: three [2][128] float regions
@@ -67,11 +71,11 @@ struct TcAttnParams {
   int32_t nodes_per_block;  // NB: nodes per 128-row tile (G * NB <= 128)
 };
 
-template <int D>
+template <int D, bool Lite = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const TcAttnParams tp) {
-  using SM = TcSmem<D>;
+  using SM = TcSmem<D, Lite>;
   constexpr int S = SM::kStages;
   const AttnParams& prm = tp.a;
   extern __shared__ uint8_t tc_smem_raw[];
@@ -104,8 +108,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int ntiles = (L + kAttnKeys - 1) / kAttnKeys;
   const int t_begin = split * prm.tiles_per_split;
   const int t_end = min(ntiles, t_begin + prm.tiles_per_split);
-  const int nt = t_end > t_begin ? t_end - t_begin : 0;
-  const bool last = split == prm.num_splits - 1;
+  int nt = t_end > t_begin ? t_end - t_begin : 0;
+  bool last = split == prm.num_splits - 1;
+  if (Lite && nt + (last ? 1 : 0) > 1) {
+    // a plan that gives a compact-layout CTA two tiles: flag it and run nothing
+    if (threadIdx.x == 0) record_error(kErrAttnPlan);
+    nt = 0;
+    last = false;
+  }
   const int T = nt + (last ? 1 : 0);  // tiles this CTA runs (prefix tiles, then the tree tile)
 
   if (threadIdx.x == 0) {
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ok = ok && mbar_wait(smem_u32(&p_full[t & 1]), (t >> 1) & 1, kErrAttnMmaWait);
         tc_fence_after();
         const uint32_t vb = (t < nt ? kv_stage(t % S) : tree_s) + SM::kTile;
-        const uint32_t pb = p_s + static_cast<uint32_t>((t & 1) * SM::kP);
+        const uint32_t pb = p_s + static_cast<uint32_t>((t % SM::kPBufs) * SM::kP);
 #pragma unroll
         for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
           const uint64_t a = smem_desc_k_sw128(pb) + 2 * kk;
@@ -327,7 +337,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;  // masked keys give exp2(-inf) = 0
       // P buffer t&1 was last read by PV(t - 2)
       if (t >= 2) mbar_wait(smem_u32(&pv_done[t & 1]), ((t - 2) >> 1) & 1, kErrAttnConsumerWait);
-      const uint32_t prow = p_s + static_cast<uint32_t>((t & 1) * SM::kP) + static_cast<uint32_t>(r * 128);
+      const uint32_t prow = p_s + static_cast<uint32_t>((t % SM::kPBufs) * SM::kP) + static_cast<uint32_t>(r * 128);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t w[4];

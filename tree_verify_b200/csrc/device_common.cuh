@@ -22,6 +22,7 @@ enum DeviceError : int32_t {
   kErrAttnProducerWait = 0x201,
   kErrAttnConsumerWait = 0x202,
   kErrAttnMmaWait = 0x203,
+  kErrAttnPlan = 0x204,       // a launch plan gave a compact-layout attention CTA two tiles
   kErrAccWait = 0x301,
   kErrAccClusterWait = 0x302,
 };

@@ -58,13 +58,18 @@ struct AttnPlan {
   int tiles_per_split;
   size_t acc_bytes;  // split partials (0 with a single split)
   size_t ml_bytes;
+  bool lite;         // one tile per CTA, compact shared-memory layout
 };
 
 // Split the prefix so that (sequences x kv heads x row blocks x splits) fills one wave of
 // one CTA per SM (the kernel's register use allows one); a split never spans more than 32
 // tiles of 64 keys.
-AttnPlan plan_attention(const eagle_shape_t* s) {
+// `lite`: one tile per CTA (the compact shared-memory layout) -- every prefix tile is a
+// split of its own and the tree tile gets one more; used where the attention runs beside
+// the LM head rather than on an idle GPU.
+AttnPlan plan_attention(const eagle_shape_t* s, bool lite = false) {
   AttnPlan p{};
+  p.lite = lite && s->dtype == EAGLE_DTYPE_BF16;
   const int G = s->num_q_heads / s->num_kv_heads;
   if (s->dtype == EAGLE_DTYPE_BF16) {
     // tensor-core path: a 128-row tile holds floor(128 / G) nodes x G heads
@@ -75,6 +80,14 @@ AttnPlan plan_attention(const eagle_shape_t* s) {
     p.row_blocks = 1;
   }
   const int max_tiles = (s->max_prefix_len + kAttnKeys - 1) / kAttnKeys;
+  if (p.lite) {
+    p.tiles_per_split = 1;
+    p.splits = max_tiles + 1;
+    const size_t rows = static_cast<size_t>(s->batch) * s->num_nodes * s->num_q_heads;
+    p.acc_bytes = align256(rows * p.splits * s->head_dim * sizeof(float));
+    p.ml_bytes = align256(rows * p.splits * 2 * sizeof(float));
+    return p;
+  }
   const long base = static_cast<long>(s->batch) * s->num_kv_heads * p.row_blocks;
   const long want = (static_cast<long>(kNumSMs) + base - 1) / base;
   int tiles_per = static_cast<int>((max_tiles + want - 1) / want);
@@ -101,7 +114,7 @@ struct LmPlan {
   size_t smem;
 };
 
-LmPlan plan_lm_head(const eagle_shape_t* s) {
+LmPlan plan_lm_head(const eagle_shape_t* s, int max_stages = 8) {
   LmPlan p{};
   const long M = static_cast<long>(s->batch) * s->num_nodes;
   p.chunks = static_cast<int>((M + 255) / 256);
@@ -114,7 +127,7 @@ LmPlan plan_lm_head(const eagle_shape_t* s) {
   } else {
     p.stages = static_cast<int>((200 * 1024) / stage);
   }
-  if (p.stages > 8) p.stages = 8;
+  if (p.stages > max_stages) p.stages = max_stages;
   if (p.stages < 2) p.stages = 2;
   int cols = 32;
   while (cols < p.bn) cols <<= 1;
@@ -152,6 +165,42 @@ AccPlan plan_accept(const eagle_shape_t* s, int max_cluster = kAccMaxCluster) {
 
 constexpr size_t kAccMaxSmem = kAccSmemBudget;
 
+// ------------------------------------------------------------------ the step's schedule
+
+// eagle_verify_step runs tree attention beside the LM head when both fit on one SM at
+// once: with a 3-stage ring the LM head (HBM-bound, two CTAs per SM) leaves room for one
+// compact-layout attention CTA, so the attention hides under the weight stream instead of
+// running after it.  Only for a single chunk of tree rows, and while the one-tile-per-CTA
+// partials stay modest.
+constexpr int kStepLmStages = 3;
+constexpr size_t kSmemPerSM = 228 * 1024;
+constexpr size_t kSmemPerCtaReserve = 1024;
+constexpr size_t kMaxOverlapWorkspace = 256ull << 20;
+
+size_t attention_ws_bytes(const eagle_shape_t* s, bool lite) {
+  const AttnPlan p = plan_attention(s, lite);
+  return p.acc_bytes + p.ml_bytes;
+}
+
+bool step_overlap(const eagle_shape_t* s);
+
+// the attention partials' share of the workspace: enough for either plan the step may take
+size_t attention_region_bytes(const eagle_shape_t* s) {
+  const size_t alone = attention_ws_bytes(s, false);
+  if (!step_overlap(s)) return alone;
+  const size_t beside = attention_ws_bytes(s, true);
+  return beside > alone ? beside : alone;
+}
+
+bool step_overlap(const eagle_shape_t* s) {
+  if (s->dtype != EAGLE_DTYPE_BF16) return false;
+  const LmPlan lm = plan_lm_head(s, kStepLmStages);
+  if (lm.chunks != 1) return false;
+  const size_t attn = s->head_dim == 64 ? TcSmem<64, true>::kAlloc : TcSmem<128, true>::kAlloc;
+  if (2 * (lm.smem + kSmemPerCtaReserve) + attn + kSmemPerCtaReserve > kSmemPerSM) return false;
+  return attention_ws_bytes(s, true) <= kMaxOverlapWorkspace;
+}
+
 // ------------------------------------------------------------------ driver entry point
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -185,6 +234,13 @@ struct DeviceState {
   std::once_flag attrs_once;
   bool attrs_ok = false;
   int max_cluster = 8;
+  // eagle_verify_step's second stream and its fork/join events, made on first use
+  std::once_flag side_once;
+  bool side_ok = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t lm_started = nullptr;
+  cudaEvent_t attn_done = nullptr;
+  std::mutex step_mu;  // one step's fork/join sequence at a time on the shared side stream
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -203,16 +259,21 @@ bool ensure_attributes(int dev) {
                                TcSmem<64>::kAlloc) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TcSmem<128>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tree_accept_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kAccMaxSmem)) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tree_accept_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kAccMaxSmem)) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               TcSmem<64, true>::kAlloc) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               TcSmem<128, true>::kAlloc) == cudaSuccess;
+    const void* walks[2] = {reinterpret_cast<const void*>(tree_accept_kernel<true>),
+                            reinterpret_cast<const void*>(tree_accept_kernel<false>)};
+    bool nonportable = true;
+    for (const void* k : walks) {
+      ok &= cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kAccMaxSmem)) == cudaSuccess;
+      nonportable &= cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    }
     // 16-CTA clusters if the device can co-schedule them, else the portable 8
     st.max_cluster = 8;
-    if (cudaFuncSetAttribute(tree_accept_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-            cudaSuccess &&
-        cudaFuncSetAttribute(tree_accept_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-            cudaSuccess) {
+    if (nonportable) {
       cudaLaunchConfig_t cfg{};
       cfg.gridDim = dim3(16);
       cfg.blockDim = dim3(kAccThreads);
@@ -234,6 +295,17 @@ bool ensure_attributes(int dev) {
   return st.attrs_ok;
 }
 
+bool ensure_side(int dev) {
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.side_once, [&] {
+    st.side_ok = cudaStreamCreateWithFlags(&st.side, cudaStreamNonBlocking) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&st.lm_started, cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&st.attn_done, cudaEventDisableTiming) == cudaSuccess;
+    cudaGetLastError();
+  });
+  return st.side_ok;
+}
+
 eagle_status_t launch_status() {
   return cudaGetLastError() == cudaSuccess ? EAGLE_OK : EAGLE_ERR_CUDA;
 }
@@ -245,7 +317,7 @@ eagle_status_t launch_status() {
 eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* kp, const void* vp,
                              const int32_t* lens, const void* kt, const void* vt,
                              const int32_t* parents, void* out, void* ws, cudaStream_t st,
-                             bool pdl = false) {
+                             bool pdl = false, bool lite = false) {
   const int B = s->batch, N = s->num_nodes, Hq = s->num_q_heads, Hkv = s->num_kv_heads;
   const int D = s->head_dim, Lmax = s->max_prefix_len;
   const float scale = softmax_scale(s);
@@ -264,7 +336,7 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
           N, Hq, Hkv, Lmax, scale);
     return launch_status();
   }
-  const AttnPlan plan = plan_attention(s);
+  const AttnPlan plan = plan_attention(s, lite);
   const int G = Hq / Hkv;
   CUtensorMap tq, tk, tv;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax),
@@ -302,15 +374,21 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(plan.row_blocks, plan.splits, B * Hkv);
   cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = D == 64 ? TcSmem<64>::kAlloc : TcSmem<128>::kAlloc;
+  cfg.dynamicSmemBytes = plan.lite ? (D == 64 ? TcSmem<64, true>::kAlloc : TcSmem<128, true>::kAlloc)
+                                   : (D == 64 ? TcSmem<64>::kAlloc : TcSmem<128>::kAlloc);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  const cudaError_t e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, tq, tk, tv, tp)
-                                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, tq, tk, tv, tp);
+  cudaError_t e;
+  if (plan.lite)
+    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64, true>, tq, tk, tv, tp)
+                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128, true>, tq, tk, tv, tp);
+  else
+    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, tq, tk, tv, tp)
+                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, tq, tk, tv, tp);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EAGLE_ERR_CUDA;
@@ -326,8 +404,10 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   return launch_status();
 }
 
+// `started`: an event that fires once every CTA has begun (the LM head's resources are
+// claimed), for a second stream to start work beside it; `max_stages` caps the TMA ring.
 eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const void* w, float* logits,
-                           cudaStream_t st) {
+                           cudaStream_t st, int max_stages = 8, cudaEvent_t started = nullptr) {
   const int M = s->batch * s->num_nodes, V = s->vocab, H = s->hidden;
   if (s->dtype == EAGLE_DTYPE_F32) {
     const dim3 grid((V + kLmF32TileV - 1) / kLmF32TileV, (M + kLmF32TileR - 1) / kLmF32TileR);
@@ -335,7 +415,7 @@ eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const voi
                                              logits, M, V, H);
     return launch_status();
   }
-  const LmPlan plan = plan_lm_head(s);
+  const LmPlan plan = plan_lm_head(s, max_stages);
   CUtensorMap tw, th;
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
   const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};
@@ -346,6 +426,25 @@ eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const voi
     return EAGLE_ERR_CUDA;
   LmTcParams prm{logits, M, V, H, plan.bn, plan.stages, plan.tmem_cols};
   const dim3 grid(plan.chunks, (V + kLmBlockV - 1) / kLmBlockV);
+  if (started != nullptr) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kLmThreads);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeLaunchCompletionEvent;
+    attr[0].val.launchCompletionEvent.event = started;
+    attr[0].val.launchCompletionEvent.flags = 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, lm_head_tc_kernel, tw, th, prm) == cudaSuccess) return launch_status();
+    // no launch-completion events here: the second stream starts after the LM head instead
+    cudaGetLastError();
+    lm_head_tc_kernel<<<grid, kLmThreads, plan.smem, st>>>(tw, th, prm);
+    if (cudaEventRecord(started, st) != cudaSuccess) return EAGLE_ERR_CUDA;
+    return launch_status();
+  }
   lm_head_tc_kernel<<<grid, kLmThreads, plan.smem, st>>>(tw, th, prm);
   return launch_status();
 }
@@ -405,7 +504,7 @@ eagle_status_t run_accept(const eagle_shape_t* s, const float* logits, const flo
 eagle_status_t check_attention_args(const eagle_shape_t* s, const void* q, const void* kp,
                                     const void* vp, const int32_t* lens, const void* kt,
                                     const void* vt, const int32_t* parents, const void* out,
-                                    const void* ws, size_t ws_bytes) {
+                                    const void* ws, size_t ws_bytes, size_t need) {
   eagle_status_t rc = check_shape(s);
   if (rc != EAGLE_OK) return rc;
   if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(kt) || !aligned16(vt) ||
@@ -413,7 +512,6 @@ eagle_status_t check_attention_args(const eagle_shape_t* s, const void* q, const
     return EAGLE_ERR_INVALID_ARGUMENT;
   if (static_cast<long>(s->batch) * s->num_kv_heads > 65535) return EAGLE_ERR_UNSUPPORTED;
   if (s->dtype == EAGLE_DTYPE_BF16 && s->num_q_heads / s->num_kv_heads > kTcRows) return EAGLE_ERR_UNSUPPORTED;
-  const size_t need = eagle_workspace_bytes(s);
   if (ws_bytes < need) return EAGLE_ERR_WORKSPACE_TOO_SMALL;
   if (need > 0 && (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0))
     return EAGLE_ERR_INVALID_ARGUMENT;
@@ -470,8 +568,7 @@ const char* eagle_status_string(eagle_status_t status) {
 
 size_t eagle_workspace_bytes(const eagle_shape_t* shape) {
   if (check_shape(shape) != EAGLE_OK) return 0;
-  const AttnPlan p = plan_attention(shape);
-  return p.acc_bytes + p.ml_bytes;
+  return attention_region_bytes(shape);
 }
 
 eagle_status_t eagle_tree_attention(const eagle_shape_t* shape, const void* q, const void* k_prefix,
@@ -479,7 +576,8 @@ eagle_status_t eagle_tree_attention(const eagle_shape_t* shape, const void* q, c
                                     const void* k_tree, const void* v_tree, const int32_t* parents,
                                     void* out, void* workspace, size_t workspace_bytes, void* stream) {
   eagle_status_t rc = check_attention_args(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
-                                           parents, out, workspace, workspace_bytes);
+                                           parents, out, workspace, workspace_bytes,
+                                           eagle_workspace_bytes(shape));
   if (rc != EAGLE_OK) return rc;
   int dev;
   if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
@@ -522,7 +620,8 @@ eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, cons
                                  int32_t* next_token, void* workspace, size_t workspace_bytes,
                                  void* stream) {
   eagle_status_t rc = check_attention_args(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
-                                           parents, out, workspace, workspace_bytes);
+                                           parents, out, workspace, workspace_bytes,
+                                           eagle_workspace_bytes(shape));
   if (rc == EAGLE_OK) rc = check_lm_args(shape, hidden, w_lm, logits);
   if (rc == EAGLE_OK)
     rc = check_accept_args(shape, logits, draft_probs, tokens, parents, temperature, accepted_nodes,
@@ -532,6 +631,32 @@ eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, cons
   if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
   if (!device_accept_supported(shape, dev)) return EAGLE_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // At T = 0 the walk is one argmax per accepted node and tree attention is the step's
+  // tail, so it moves beside the LM head; at T > 0 the walk outlasts the attention that
+  // follows the LM head, and the LM head runs alone at full depth.
+  const bool overlap = temperature == 0.f && step_overlap(shape) &&
+                       workspace_bytes >= attention_ws_bytes(shape, true) && ensure_side(dev);
+  if (overlap) {
+    // Two streams: the LM head streams W over the whole GPU; once all of its CTAs hold
+    // their SMs, tree attention (compact layout, one tile per CTA) and its merge start on
+    // the side stream in the room they leave; the accept walk follows the LM head on the
+    // caller's stream (programmatic dependent launch), and the caller's stream then waits
+    // for the attention.
+    DeviceState& ds = g_dev[dev];
+    std::lock_guard<std::mutex> lock(ds.step_mu);
+    rc = run_lm_head(shape, hidden, w_lm, logits, st, kStepLmStages, ds.lm_started);
+    if (rc != EAGLE_OK) return rc;
+    if (cudaStreamWaitEvent(ds.side, ds.lm_started, 0) != cudaSuccess) return EAGLE_ERR_CUDA;
+    rc = run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
+                       workspace, ds.side, /*pdl=*/false, /*lite=*/true);
+    if (rc != EAGLE_OK) return rc;
+    if (cudaEventRecord(ds.attn_done, ds.side) != cudaSuccess) return EAGLE_ERR_CUDA;
+    rc = run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed, offset,
+                    accepted_nodes, accept_len, next_token, st, /*pdl=*/true);
+    if (rc != EAGLE_OK) return rc;
+    if (cudaStreamWaitEvent(st, ds.attn_done, 0) != cudaSuccess) return EAGLE_ERR_CUDA;
+    return EAGLE_OK;
+  }
   // One stream, three overlapping phases: the LM head streams W over the whole GPU; the
   // accept walk (programmatic dependent launch) sets up while the LM head drains and walks
   // on one cluster per sequence; tree attention (its output does not feed the walk) is
@@ -594,13 +719,14 @@ extern "C" eagle_status_t eagle_tree_attention_static(const eagle_shape_t* shape
                                                       const void* v_tree, const int32_t* parents,
                                                       void* out, void* stream) {
   if (check_shape(shape) != EAGLE_OK) return EAGLE_ERR_INVALID_ARGUMENT;
-  if (eagle_workspace_bytes(shape) > EAGLE_STATIC_SCRATCH_BYTES) return EAGLE_ERR_UNSUPPORTED;
+  if (attention_ws_bytes(shape, false) > EAGLE_STATIC_SCRATCH_BYTES) return EAGLE_ERR_UNSUPPORTED;
   int dev;
   if (!current_device(&dev)) return EAGLE_ERR_CUDA;
   void* scratch = static_scratch_address(dev);
   if (scratch == nullptr) return EAGLE_ERR_CUDA;
   eagle_status_t rc = check_attention_args(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
-                                           parents, out, scratch, EAGLE_STATIC_SCRATCH_BYTES);
+                                           parents, out, scratch, EAGLE_STATIC_SCRATCH_BYTES,
+                                           attention_ws_bytes(shape, false));
   if (rc != EAGLE_OK) return rc;
   if (!ensure_attributes(dev)) return EAGLE_ERR_CUDA;
   return run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,

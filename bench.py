@@ -43,6 +43,22 @@ def _peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def _lm_head_traffic(workload: str):
+    """DRAM bytes per LM-head launch from the committed ncu capture of this workload, or
+    None when there is none or the kernel's sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"lm_head_tc_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    for rel, digest in rec["sources_sha256"].items():
+        with open(os.path.join(ROOT, rel), "rb") as src:
+            if hashlib.sha256(src.read()).hexdigest() != digest:
+                return None
+    return int(rec["traffic_bytes_per_launch"])
+
+
 def step_bytes(w, prefix_lens):
     el = 2 if w.dtype == wl.BF16 else 4
     B, N, Hq, Hkv, D, H, V = (w.batch, w.num_nodes, w.num_q_heads, w.num_kv_heads, w.head_dim,
@@ -315,7 +331,7 @@ def main():
         "step_ms_p10_p50_p90": [float(np.percentile(step_ms, q)) for q in (10, 50, 90)],
         "roofline": {"kernel": "lm_head_tc_kernel", "bound": "hbm", "achieved": lm_gbs,
                      "peak": peak, "unit": "GB/s", "frac": lm_gbs / peak,
-                     "traffic": None, "bytes_per_launch": nb["lm_head"],
+                     "traffic": _lm_head_traffic(w.name), "bytes_per_launch": nb["lm_head"],
                      "us_per_launch": lm_ms * 1e3, "peak_kind": peak_kind},
         "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "verify-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

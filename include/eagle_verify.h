@@ -146,18 +146,19 @@ eagle_status_t eagle_tree_accept(const eagle_shape_t *shape, const float *logits
                                  void *stream);
 
 /*
- * One whole verification step: LM-head logits, the accept walk and tree attention,
- * enqueued on `stream` in that order.  The walk may begin while the LM head drains and
- * waits for it before reading the logits; tree attention, whose output the walk does not
- * read, may run while the walk runs.  Arguments as above; writes out, logits,
- * accepted_nodes, accept_len and next_token.
+ * One whole verification step: LM-head logits, the accept walk and tree attention.
+ * Arguments as above; writes out, logits, accepted_nodes, accept_len and next_token.
+ * The LM head and then the walk are enqueued on `stream`; the walk may begin while the LM
+ * head drains and waits for it before reading the logits.
  *
- * Greedy steps (temperature 0) on bf16 shapes with few tree rows (B*N <= 48 at D = 128)
- * instead run tree attention beside the LM head: the library enqueues it on a second
- * stream of its own (one per device, created with two events on the first such call) that
- * starts once the LM head's CTAs hold their SMs, and `stream` waits for it before any work
- * enqueued after this call.  Such calls on one device are serialised on the host while
- * they are enqueued.  The workspace from eagle_workspace_bytes() covers both schedules.
+ * bf16: tree attention (whose output the walk does not read) and its split merge run on a
+ * second stream of the library's own (one per device, created with two events on the first
+ * bf16 call), and `stream` waits for them before any work enqueued after this call.  The
+ * attention starts when the LM head completes and runs while the walk runs; greedy steps
+ * (temperature 0) on shapes with few tree rows (B*N <= 48 at D = 128) start it beside the
+ * LM head instead, once every LM-head CTA holds its SM.  bf16 calls on one device are
+ * serialised on the host while they are enqueued.  fp32: everything on `stream`, tree
+ * attention after the walk.  The workspace from eagle_workspace_bytes() covers both plans.
  */
 eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
                                  const void *k_prefix, const void *v_prefix,

@@ -238,7 +238,7 @@ struct DeviceState {
   std::once_flag side_once;
   bool side_ok = false;
   cudaStream_t side = nullptr;
-  cudaEvent_t lm_started = nullptr;
+  cudaEvent_t lm_mark = nullptr;  // LM head under way (T = 0 beside it) or completed
   cudaEvent_t attn_done = nullptr;
   std::mutex step_mu;  // one step's fork/join sequence at a time on the shared side stream
 };
@@ -299,7 +299,7 @@ bool ensure_side(int dev) {
   DeviceState& st = g_dev[dev];
   std::call_once(st.side_once, [&] {
     st.side_ok = cudaStreamCreateWithFlags(&st.side, cudaStreamNonBlocking) == cudaSuccess &&
-                 cudaEventCreateWithFlags(&st.lm_started, cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&st.lm_mark, cudaEventDisableTiming) == cudaSuccess &&
                  cudaEventCreateWithFlags(&st.attn_done, cudaEventDisableTiming) == cudaSuccess;
     cudaGetLastError();
   });
@@ -312,12 +312,11 @@ eagle_status_t launch_status() {
 
 // ------------------------------------------------------------------ launches
 
-// `pdl`: launched right behind the accept walk of the same step, whose outputs it does not
-// read; it may then start while the walk is still running.
+// `lite`: the one-tile-per-CTA plan and compact layout (the step's greedy schedule).
 eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* kp, const void* vp,
                              const int32_t* lens, const void* kt, const void* vt,
                              const int32_t* parents, void* out, void* ws, cudaStream_t st,
-                             bool pdl = false, bool lite = false) {
+                             bool lite = false) {
   const int B = s->batch, N = s->num_nodes, Hq = s->num_q_heads, Hkv = s->num_kv_heads;
   const int D = s->head_dim, Lmax = s->max_prefix_len;
   const float scale = softmax_scale(s);
@@ -377,11 +376,6 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   cfg.dynamicSmemBytes = plan.lite ? (D == 64 ? TcSmem<64, true>::kAlloc : TcSmem<128, true>::kAlloc)
                                    : (D == 64 ? TcSmem<64>::kAlloc : TcSmem<128>::kAlloc);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
   cudaError_t e;
   if (plan.lite)
     e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64, true>, tq, tk, tv, tp)
@@ -631,24 +625,27 @@ eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, cons
   if (!current_device(&dev) || !ensure_attributes(dev)) return EAGLE_ERR_CUDA;
   if (!device_accept_supported(shape, dev)) return EAGLE_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // At T = 0 the walk is one argmax per accepted node and tree attention is the step's
-  // tail, so it moves beside the LM head; at T > 0 the walk outlasts the attention that
-  // follows the LM head, and the LM head runs alone at full depth.
-  const bool overlap = temperature == 0.f && step_overlap(shape) &&
-                       workspace_bytes >= attention_ws_bytes(shape, true) && ensure_side(dev);
-  if (overlap) {
-    // Two streams: the LM head streams W over the whole GPU; once all of its CTAs hold
-    // their SMs, tree attention (compact layout, one tile per CTA) and its merge start on
-    // the side stream in the room they leave; the accept walk follows the LM head on the
-    // caller's stream (programmatic dependent launch), and the caller's stream then waits
-    // for the attention.
+  if (shape->dtype == EAGLE_DTYPE_BF16 && ensure_side(dev)) {
+    // Two streams.  The LM head streams W over the whole GPU and the accept walk follows it
+    // on the caller's stream (programmatic dependent launch: the walk's set-up overlaps the
+    // LM head's drain).  Tree attention, whose output the walk does not read, runs with its
+    // merge on a library-owned side stream, and the caller's stream waits for it after the
+    // walk.  Greedy steps on shapes with few tree rows start it beside the LM head (compact
+    // layout, one tile per CTA) once every LM-head CTA holds its SM: there the walk is one
+    // argmax per accepted node and the attention would be the step's tail.  Otherwise it
+    // starts when the LM head completes and runs while the walk runs.  No kernel is ever
+    // launched as a programmatic dependent of the walk.
     DeviceState& ds = g_dev[dev];
     std::lock_guard<std::mutex> lock(ds.step_mu);
-    rc = run_lm_head(shape, hidden, w_lm, logits, st, kStepLmStages, ds.lm_started);
+    const bool beside = temperature == 0.f && step_overlap(shape) &&
+                        workspace_bytes >= attention_ws_bytes(shape, true);
+    rc = run_lm_head(shape, hidden, w_lm, logits, st, beside ? kStepLmStages : 8,
+                     beside ? ds.lm_mark : nullptr);
     if (rc != EAGLE_OK) return rc;
-    if (cudaStreamWaitEvent(ds.side, ds.lm_started, 0) != cudaSuccess) return EAGLE_ERR_CUDA;
+    if (!beside && cudaEventRecord(ds.lm_mark, st) != cudaSuccess) return EAGLE_ERR_CUDA;
+    if (cudaStreamWaitEvent(ds.side, ds.lm_mark, 0) != cudaSuccess) return EAGLE_ERR_CUDA;
     rc = run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
-                       workspace, ds.side, /*pdl=*/false, /*lite=*/true);
+                       workspace, ds.side, /*lite=*/beside);
     if (rc != EAGLE_OK) return rc;
     if (cudaEventRecord(ds.attn_done, ds.side) != cudaSuccess) return EAGLE_ERR_CUDA;
     rc = run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed, offset,
@@ -657,17 +654,15 @@ eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, cons
     if (cudaStreamWaitEvent(st, ds.attn_done, 0) != cudaSuccess) return EAGLE_ERR_CUDA;
     return EAGLE_OK;
   }
-  // One stream, three overlapping phases: the LM head streams W over the whole GPU; the
-  // accept walk (programmatic dependent launch) sets up while the LM head drains and walks
-  // on one cluster per sequence; tree attention (its output does not feed the walk) is
-  // released by the walk and fills the SMs the walk leaves idle.
+  // fp32 (and bf16 if the side stream could not be made): one stream -- the LM head, the
+  // walk (programmatic dependent launch), then tree attention once the walk has completed
   rc = run_lm_head(shape, hidden, w_lm, logits, st);
   if (rc != EAGLE_OK) return rc;
   rc = run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed, offset,
                   accepted_nodes, accept_len, next_token, st, /*pdl=*/true);
   if (rc != EAGLE_OK) return rc;
   return run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
-                       workspace, st, /*pdl=*/true);
+                       workspace, st);
 }
 
 eagle_status_t eagle_device_error(int32_t* code, int32_t reset) {

@@ -11,6 +11,8 @@ Functions (each follows the passage cited in ``oracle.c``):
   lm_head         O2 -- logits = hidden W^T (EAGLE summary, section 3 "Draft model")
   tree_accept     O3 -- multi-round speculative sampling walk (EAGLE summary, section 2,
                         appendix A.2 and appendix B "Algorithm 1")
+  commit          O4 -- append the root and the accepted nodes to the prefix K/V cache and
+                        gather their hidden rows (EAGLE summary, section 3)
   race, uniform, philox -- the sampler and the counter-based generator it uses
 """
 from __future__ import annotations
@@ -58,6 +60,8 @@ def lib() -> ctypes.CDLL:
                                          ctypes.c_double, ctypes.c_int, vp, vp]
         L.orc_lm_head.argtypes = [ctypes.c_int] * 4 + [vp, vp, ctypes.c_int, vp, vp]
         L.orc_lm_head.restype = None
+        L.orc_commit.restype = None
+        L.orc_commit.argtypes = [ctypes.c_int] * 7 + [vp] * 11
         L.orc_race.restype = ctypes.c_int32
         L.orc_race.argtypes = [ctypes.c_int, vp, ctypes.c_uint64, ctypes.c_uint64,
                                ctypes.c_int32, ctypes.c_int32, vp]
@@ -196,3 +200,31 @@ def tree_accept(draft_probs, tokens, parents, temperature: float, seed: int = 0,
         raise ValueError(f"oracle tree_accept rejected its inputs (code {rc})")
     return dict(accepted_nodes=acc, accept_len=alen, next_token=nxt, near=near,
                 decisions=ndec, first_near=first)
+
+
+def commit(k_prefix, v_prefix, prefix_lens, k_tree, v_tree, hidden, parents, accepted_nodes,
+           accept_len, feat=None):
+    """O4: the post-accept commit on copies of the cache (bit-for-bit element copies).
+
+    k_prefix/v_prefix [B, Hkv, Lmax, D], k_tree/v_tree [B, N, Hkv, D], hidden [B, N, H]
+    (all of one element type: uint16 bf16 bits or float32), parents / accepted_nodes [B, N]
+    and prefix_lens / accept_len [B] int32.  feat [B, N, H] gives the rows the commit does not
+    write (default zeros).  Returns (k_prefix', v_prefix', new_lens, feat')."""
+    kp = np.ascontiguousarray(k_prefix).copy()
+    vp = np.ascontiguousarray(v_prefix).copy()
+    B, Hkv, Lmax, D = kp.shape
+    N = k_tree.shape[1]
+    H = hidden.shape[-1]
+    kt = np.ascontiguousarray(k_tree, dtype=kp.dtype)
+    vt = np.ascontiguousarray(v_tree, dtype=kp.dtype)
+    hid = np.ascontiguousarray(hidden, dtype=kp.dtype)
+    out = (np.zeros((B, N, H), kp.dtype) if feat is None
+           else np.ascontiguousarray(feat, dtype=kp.dtype).copy())
+    lens = np.ascontiguousarray(prefix_lens, np.int32)
+    par = np.ascontiguousarray(parents, np.int32)
+    acc = np.ascontiguousarray(accepted_nodes, np.int32)
+    alen = np.ascontiguousarray(accept_len, np.int32)
+    new = np.empty(B, np.int32)
+    lib().orc_commit(B, N, Hkv, D, Lmax, H, kp.itemsize, _p(kp), _p(vp), _p(lens), _p(kt), _p(vt),
+                     _p(hid), _p(par), _p(acc), _p(alen), _p(new), _p(out))
+    return kp, vp, new, out

@@ -25,6 +25,13 @@
  *                        adjusted distribution; appendix B: Algorithm 1 takes the
  *                        target distribution, the candidates and their own
  *                        distributions and returns one sample of the target).
+ *   O4 commit           (EAGLE summary, section 3 "Drafting and verification": the
+ *                        accepted draft tokens extend the target's context, and
+ *                        the features of the accepted tokens feed the next
+ *                        drafting round): the root and the accepted nodes, in
+ *                        root-to-leaf order, are appended to the prefix K/V cache
+ *                        and their hidden rows gathered, as sequential decoding of
+ *                        those tokens would have left the cache.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - the adjusted distribution is norm(max(0, p - p_hat)) (standard speculative
@@ -459,6 +466,61 @@ int orc_tree_accept(int B, int N, int V, int logits_mode, const void *logits, in
         free(r);
     }
     return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ O4 commit */
+
+/* Post-accept commit of one step.  For sequence b with a = accept_len[b] >= 0 the
+ * committed path is node 0 (the root: the token committed by the previous step, whose K/V
+ * this step computed as a tree row) followed by accepted_nodes[b][0 .. a-1]; n = a + 1.
+ * Row t of the path goes to position L_b + t of every kv head of the prefix cache
+ * (k_prefix/v_prefix [B, Hkv, Lmax, D], elements of `esize` bytes, copied bit for bit)
+ * and to row t of feat [B, N, H] (from hidden [B*N, H]); new_lens[b] = L_b + n.  Nothing
+ * is written for the sequence and new_lens[b] is
+ *   L_b  when a == -1 (the walk found the tree invalid);
+ *   -1   when a is out of [-1, N-1], L_b out of [0, Lmax], L_b + n > Lmax, or the path is
+ *        not a root-to-leaf chain of the tree (node t+1 a child of node t).
+ * feat rows n .. N-1 and cache positions outside [L_b, L_b + n) are left as they are. */
+void orc_commit(int B, int N, int Hkv, int D, int Lmax, int H, int esize,
+                void *k_prefix, void *v_prefix, const int32_t *prefix_lens,
+                const void *k_tree, const void *v_tree, const void *hidden,
+                const int32_t *parents, const int32_t *accepted_nodes, const int32_t *accept_len,
+                int32_t *new_lens, void *feat)
+{
+    const size_t row = (size_t)D * esize, hrow = (size_t)H * esize;
+    for (int b = 0; b < B; ++b) {
+        const int32_t L = prefix_lens[b], a = accept_len[b];
+        const int32_t *acc = accepted_nodes + (size_t)b * N;
+        const int32_t *par = parents + (size_t)b * N;
+        if (a == -1) {
+            new_lens[b] = L;
+            continue;
+        }
+        int ok = a >= 0 && a <= N - 1 && L >= 0 && L <= Lmax && L + a + 1 <= Lmax;
+        int path[64];
+        path[0] = 0;
+        for (int t = 1; ok && t <= a; ++t) {
+            const int32_t c = acc[t - 1];
+            ok = c >= 1 && c < N && par[c] == path[t - 1];
+            path[t] = c;
+        }
+        if (!ok) {
+            new_lens[b] = -1;
+            continue;
+        }
+        const int n = a + 1;
+        for (int t = 0; t < n; ++t) {
+            const size_t node = (size_t)b * N + path[t];
+            for (int g = 0; g < Hkv; ++g) {
+                const size_t src = (node * Hkv + g) * row;
+                const size_t dst = (((size_t)b * Hkv + g) * Lmax + L + t) * row;
+                memcpy((char *)k_prefix + dst, (const char *)k_tree + src, row);
+                memcpy((char *)v_prefix + dst, (const char *)v_tree + src, row);
+            }
+            memcpy((char *)feat + ((size_t)b * N + t) * hrow, (const char *)hidden + node * hrow, hrow);
+        }
+        new_lens[b] = L + n;
+    }
 }
 
 /* Uniforms U(b, node, v, purpose) for v = 0..n-1 (test helper for the generator pins). */

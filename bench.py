@@ -280,6 +280,30 @@ def main():
     barrier()
     lm_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(ls, le)]))
 
+    # ---- the post-accept commit of the last step's walk (timed on its own, not part of the
+    # step): the root and accepted nodes into a cache with room for them, L2 flushed first
+    B, N, Hkv, D, H = w.batch, w.num_nodes, w.num_kv_heads, w.head_dim, w.hidden
+    k_cache = torch.zeros((B, Hkv, w.prefix_len + N, D), dtype=x.k_prefix.dtype, device=dev)
+    v_cache = torch.zeros_like(k_cache)
+    new_lens = torch.empty((B,), dtype=torch.int32, device=dev)
+    feat = torch.empty((B, N, H), dtype=x.hidden.dtype, device=dev)
+    cs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ce = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        l2_flush()
+        cs[i].record(stream)
+        step.commit(x, k_cache, v_cache, new_lens, feat)
+        ce[i].record(stream)
+    barrier()
+    commit_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(cs, ce)]))
+    assert binding.device_error(reset=True) == 0
+    alen = step.accept_len.cpu().numpy()
+    commit_rows = int(np.sum(alen[alen >= 0] + 1))
+    el = x.k_prefix.element_size()
+    # each committed row: K and V of every kv head and one hidden row, read once, written once
+    commit_bytes = commit_rows * (Hkv * D * el * 2 + H * el) * 2
+
     # ---- end to end through the public API with host buffers: per-step tree inputs
     # (queries, tree K/V, hidden states, parents, tokens, draft distributions) copied from
     # pinned host memory, the walk's results read back; the prefix K/V cache and W stay
@@ -307,7 +331,7 @@ def main():
     assert binding.device_error(reset=True) == 0
 
     # ---- max over ranks
-    total_ms, e2e_ms, lm_ms = max_over_ranks([total_ms, e2e_ms, lm_ms], dist, dev)
+    total_ms, e2e_ms, lm_ms, commit_ms = max_over_ranks([total_ms, e2e_ms, lm_ms, commit_ms], dist, dev)
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -333,6 +357,10 @@ def main():
                      "peak": peak, "unit": "GB/s", "frac": lm_gbs / peak,
                      "traffic": _lm_head_traffic(w.name), "bytes_per_launch": nb["lm_head"],
                      "us_per_launch": lm_ms * 1e3, "peak_kind": peak_kind},
+        "commit": {"kernel": "commit_kernel", "us_per_launch": commit_ms * 1e3,
+                   "rows": commit_rows, "bytes_per_launch": commit_bytes,
+                   "achieved_gbs": commit_bytes / (commit_ms / 1e3) / 1e9,
+                   "frac": commit_bytes / (commit_ms / 1e3) / 1e9 / peak, "bound": "latency"},
         "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "verify-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -347,6 +375,22 @@ def main():
         result["cpu_baseline"] = {"value": 1.0 / float(np.mean(secs)), "unit": "verify-steps/s",
                                   "cores": cores, "kind": "oracle",
                                   "sample": f"{len(secs)} x [{label}]"}
+        # the oracle's commit of the same accepted nodes (it copies the whole cache first)
+        import oracle
+        acc_h = step.accepted_nodes.cpu().numpy()
+        hid = inp["hidden"].reshape(B, N, H)
+        kc, vc = k_cache.cpu(), v_cache.cpu()
+        if kc.dtype == torch.bfloat16:
+            kc, vc = kc.view(torch.int16).numpy().view(np.uint16), vc.view(torch.int16).numpy().view(np.uint16)
+        else:
+            kc, vc = kc.numpy(), vc.numpy()
+        t0 = time.perf_counter()
+        reps = 0
+        while reps < 3 or time.perf_counter() - t0 < 1.0:
+            oracle.commit(kc, vc, inp["prefix_lens"], inp["k_tree"], inp["v_tree"], hid,
+                          inp["parents"], acc_h, alen)
+            reps += 1
+        result["commit"]["oracle_us"] = (time.perf_counter() - t0) / reps * 1e6
     print(json.dumps(result))
     if dist is not None:
         dist.destroy_process_group()

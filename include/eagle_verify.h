@@ -201,6 +201,38 @@ eagle_status_t eagle_tree_attention_static(const eagle_shape_t *shape, const voi
                                            void *out, void *stream);
 
 /*
+ * Post-accept commit (EAGLE summary, section 3 "Drafting and verification": the accepted
+ * draft tokens extend the target's context, and the features of the accepted tokens feed
+ * the next drafting round).  For sequence b with a = accept_len[b] >= 0 the committed path
+ * is node 0 (the root, committed by the previous step; this step computed its K/V as a tree
+ * row) followed by accepted_nodes[b][0 .. a-1]: n = a + 1 rows, root first, and
+ *     k_prefix[b, g, L_b + t, :] = k_tree[b, path[t], g, :]   (v likewise)  t < n, every g
+ *     feat[b, t, :]              = hidden[b*N + path[t], :]
+ *     new_prefix_lens[b]         = L_b + n
+ * with L_b = prefix_lens[b]; every element is copied bit for bit, as sequential decoding of
+ * those tokens would have left the cache.  Errors only the device can see write nothing for
+ * that sequence and set new_prefix_lens[b] to
+ *     L_b  when a == -1 (eagle_tree_accept found the tree invalid);
+ *     -1   when a < -1 or a > N-1, L_b is outside [0, Lmax], L_b + n > Lmax, or the path is
+ *          not a chain of `parents` from the root.
+ *   k_prefix, v_prefix  [B, Hkv, Lmax, D] dtype; written only at positions [L_b, L_b + n)
+ *   prefix_lens         [B] int32 device; must not overlap new_prefix_lens
+ *   k_tree, v_tree      [B, N, Hkv, D] dtype
+ *   hidden              [B*N, H] dtype (the LM head's input)
+ *   parents             [B, N] int32
+ *   accepted_nodes      [B, N] int32, accept_len [B] int32 (eagle_tree_accept's outputs)
+ *   new_prefix_lens     [B] int32 out
+ *   feat                [B, N, H] dtype out; rows n .. N-1 are left as they are
+ * Takes no workspace and allocates nothing.
+ */
+eagle_status_t eagle_commit_accepted(const eagle_shape_t *shape, void *k_prefix, void *v_prefix,
+                                     const int32_t *prefix_lens, const void *k_tree,
+                                     const void *v_tree, const void *hidden,
+                                     const int32_t *parents, const int32_t *accepted_nodes,
+                                     const int32_t *accept_len, int32_t *new_prefix_lens,
+                                     void *feat, void *stream);
+
+/*
  * Reads (and, if `reset` != 0, clears) the device error word that bounded waits set
  * when they give up.  Synchronises the current device.  *code = 0 means no error.
  */

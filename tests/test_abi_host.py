@@ -127,6 +127,22 @@ def test_verify_step_validates_every_stage(lib):
     del common
 
 
+def test_commit_checks_arguments_before_launch(lib):
+    s = _shape()
+    args = [FAKE, FAKE, FAKE + 4096, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8192, FAKE]
+    bad = list(args)
+    bad[0] = None  # k_prefix
+    assert lib.eagle_commit_accepted(ctypes.byref(s), *bad, None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    bad = list(args)
+    bad[5] = FAKE + 8  # misaligned hidden
+    assert lib.eagle_commit_accepted(ctypes.byref(s), *bad, None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    bad = list(args)
+    bad[9] = args[2] + 2  # new_prefix_lens overlaps prefix_lens
+    assert lib.eagle_commit_accepted(ctypes.byref(s), *bad, None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    s_bad = _shape(num_nodes=65)
+    assert lib.eagle_commit_accepted(ctypes.byref(s_bad), *args, None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "nope.so"))
     monkeypatch.setattr(binding, "_lib", None)

@@ -23,7 +23,7 @@ DTYPE_BF16 = 1
 
 EXPORTED = ("eagle_status_string", "eagle_workspace_bytes", "eagle_tree_attention",
             "eagle_lm_head_logits", "eagle_tree_accept", "eagle_verify_step",
-            "eagle_device_error")
+            "eagle_commit_accepted", "eagle_device_error")
 
 
 class Shape(ctypes.Structure):
@@ -75,6 +75,8 @@ def load() -> ctypes.CDLL:
     L.eagle_tree_accept.argtypes = [sp, vp, vp, vp, vp, f32, u64, u64, vp, vp, vp, vp, sz, vp]
     L.eagle_verify_step.restype = ctypes.c_int
     L.eagle_verify_step.argtypes = ([sp] + [vp] * 11 + [f32, u64, u64] + [vp] * 6 + [sz, vp])
+    L.eagle_commit_accepted.restype = ctypes.c_int
+    L.eagle_commit_accepted.argtypes = [sp] + [vp] * 12
     L.eagle_device_error.restype = ctypes.c_int
     L.eagle_device_error.argtypes = [ctypes.POINTER(i32), i32]
     _lib = L
@@ -152,6 +154,14 @@ def verify_step(shape: Shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree
         _ptr(tokens), float(temperature), int(seed), int(offset), _ptr(out), _ptr(logits),
         _ptr(accepted_nodes), _ptr(accept_len), _ptr(next_token), _ptr(workspace),
         _nbytes(workspace), _stream(stream)))
+
+
+def commit_accepted(shape: Shape, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, hidden, parents,
+                    accepted_nodes, accept_len, new_prefix_lens, feat, stream=None) -> None:
+    _check("eagle_commit_accepted", load().eagle_commit_accepted(
+        ctypes.byref(shape), _ptr(k_prefix), _ptr(v_prefix), _ptr(prefix_lens), _ptr(k_tree),
+        _ptr(v_tree), _ptr(hidden), _ptr(parents), _ptr(accepted_nodes), _ptr(accept_len),
+        _ptr(new_prefix_lens), _ptr(feat), _stream(stream)))
 
 
 def device_error(reset: bool = True) -> int:

@@ -15,6 +15,7 @@
 #include "accept.cuh"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "commit.cuh"
 #include "device_common.cuh"
 #include "lm_head.cuh"
 
@@ -493,6 +494,33 @@ eagle_status_t run_accept(const eagle_shape_t* s, const float* logits, const flo
   return launch_status();
 }
 
+eagle_status_t run_commit(const eagle_shape_t* s, void* kp, void* vp, const int32_t* lens,
+                          const void* kt, const void* vt, const void* hidden, const int32_t* parents,
+                          const int32_t* acc, const int32_t* alen, int32_t* new_lens, void* feat,
+                          cudaStream_t st) {
+  const int esize = s->dtype == EAGLE_DTYPE_BF16 ? 2 : 4;
+  CommitParams p{};
+  p.k_prefix = static_cast<uint8_t*>(kp);
+  p.v_prefix = static_cast<uint8_t*>(vp);
+  p.prefix_lens = lens;
+  p.k_tree = static_cast<const uint8_t*>(kt);
+  p.v_tree = static_cast<const uint8_t*>(vt);
+  p.hidden = static_cast<const uint8_t*>(hidden);
+  p.parents = parents;
+  p.accepted_nodes = acc;
+  p.accept_len = alen;
+  p.new_lens = new_lens;
+  p.feat = static_cast<uint8_t*>(feat);
+  p.N = s->num_nodes;
+  p.Hkv = s->num_kv_heads;
+  p.Lmax = s->max_prefix_len;
+  p.row_bytes = s->head_dim * esize;
+  p.hrow_bytes = s->hidden * esize;
+  const dim3 grid(s->batch, s->num_kv_heads + s->num_nodes);
+  commit_kernel<<<grid, kCommitThreads, 0, st>>>(p);
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ argument checks
 
 eagle_status_t check_attention_args(const eagle_shape_t* s, const void* q, const void* kp,
@@ -533,6 +561,24 @@ eagle_status_t check_accept_args(const eagle_shape_t* s, const float* logits, co
   // checks the current device before anything is enqueued
   const AccPlan ap = plan_accept(s, kAccMaxCluster);
   if (ap.nq < 1 || ap.smem > kAccMaxSmem) return EAGLE_ERR_UNSUPPORTED;
+  return EAGLE_OK;
+}
+
+eagle_status_t check_commit_args(const eagle_shape_t* s, const void* kp, const void* vp,
+                                 const int32_t* lens, const void* kt, const void* vt,
+                                 const void* hidden, const int32_t* parents, const int32_t* acc,
+                                 const int32_t* alen, const int32_t* new_lens, const void* feat) {
+  eagle_status_t rc = check_shape(s);
+  if (rc != EAGLE_OK) return rc;
+  if (!aligned16(kp) || !aligned16(vp) || !aligned16(kt) || !aligned16(vt) || !aligned16(hidden) ||
+      !aligned16(feat) || lens == nullptr || parents == nullptr || acc == nullptr ||
+      alen == nullptr || new_lens == nullptr)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  // the kernel reads prefix_lens[b] in every block while one block writes new_lens[b]
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(lens), b0 = reinterpret_cast<uintptr_t>(new_lens);
+  const uintptr_t span = static_cast<uintptr_t>(s->batch) * sizeof(int32_t);
+  if (a0 < b0 + span && b0 < a0 + span) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (s->num_kv_heads + s->num_nodes > 65535) return EAGLE_ERR_UNSUPPORTED;
   return EAGLE_OK;
 }
 
@@ -663,6 +709,19 @@ eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, cons
   if (rc != EAGLE_OK) return rc;
   return run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
                        workspace, st);
+}
+
+eagle_status_t eagle_commit_accepted(const eagle_shape_t* shape, void* k_prefix, void* v_prefix,
+                                     const int32_t* prefix_lens, const void* k_tree,
+                                     const void* v_tree, const void* hidden, const int32_t* parents,
+                                     const int32_t* accepted_nodes, const int32_t* accept_len,
+                                     int32_t* new_prefix_lens, void* feat, void* stream) {
+  const eagle_status_t rc = check_commit_args(shape, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
+                                              hidden, parents, accepted_nodes, accept_len,
+                                              new_prefix_lens, feat);
+  if (rc != EAGLE_OK) return rc;
+  return run_commit(shape, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, hidden, parents,
+                    accepted_nodes, accept_len, new_prefix_lens, feat, static_cast<cudaStream_t>(stream));
 }
 
 eagle_status_t eagle_device_error(int32_t* code, int32_t reset) {

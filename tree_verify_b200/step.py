@@ -80,6 +80,20 @@ class VerifyStep:
                             self.accept_len, self.next_token, self.workspace, stream)
 
 
+    def commit(self, x: StepInputs, k_cache: torch.Tensor, v_cache: torch.Tensor,
+               new_prefix_lens: torch.Tensor, feat: torch.Tensor, stream=None) -> None:
+        """Post-accept commit of this step's walk: the root and the accepted nodes' K/V into
+        k_cache/v_cache [B, Hkv, Lcap, D] at prefix_lens.. (Lcap from the cache's shape), their
+        hidden rows into feat [B, N, H], the new lengths into new_prefix_lens [B]."""
+        s = self.shape
+        cache_shape = binding.make_shape(s.batch, s.num_nodes, s.num_q_heads, s.num_kv_heads,
+                                         s.head_dim, k_cache.shape[2], s.hidden, s.vocab, s.dtype,
+                                         s.softmax_scale)
+        binding.commit_accepted(cache_shape, k_cache, v_cache, x.prefix_lens, x.k_tree, x.v_tree,
+                                x.hidden, x.parents, self.accepted_nodes, self.accept_len,
+                                new_prefix_lens, feat, stream)
+
+
 def shape_from_workload(w) -> binding.Shape:
     return binding.make_shape(w.batch, w.num_nodes, w.num_q_heads, w.num_kv_heads, w.head_dim,
                               w.prefix_len, w.hidden, w.vocab, w.dtype)

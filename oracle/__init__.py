@@ -13,6 +13,8 @@ Functions (each follows the passage cited in ``oracle.c``):
                         appendix A.2 and appendix B "Algorithm 1")
   commit          O4 -- append the root and the accepted nodes to the prefix K/V cache and
                         gather their hidden rows (EAGLE summary, section 3)
+  tree_rerank     O5 -- the m candidates with the highest path confidence, renumbered as a
+                        tree (EAGLE-2 blog, sections 1 and 4)
   race, uniform, philox -- the sampler and the counter-based generator it uses
 """
 from __future__ import annotations
@@ -60,6 +62,8 @@ def lib() -> ctypes.CDLL:
                                          ctypes.c_double, ctypes.c_int, vp, vp]
         L.orc_lm_head.argtypes = [ctypes.c_int] * 4 + [vp, vp, ctypes.c_int, vp, vp]
         L.orc_lm_head.restype = None
+        L.orc_tree_rerank.restype = None
+        L.orc_tree_rerank.argtypes = [ctypes.c_int] * 3 + [vp] * 8
         L.orc_commit.restype = None
         L.orc_commit.argtypes = [ctypes.c_int] * 7 + [vp] * 11
         L.orc_race.restype = ctypes.c_int32
@@ -228,3 +232,20 @@ def commit(k_prefix, v_prefix, prefix_lens, k_tree, v_tree, hidden, parents, acc
     lib().orc_commit(B, N, Hkv, D, Lmax, H, kp.itemsize, _p(kp), _p(vp), _p(lens), _p(kt), _p(vt),
                      _p(hid), _p(par), _p(acc), _p(alen), _p(new), _p(out))
     return kp, vp, new, out
+
+
+def tree_rerank(parents, tokens, confidence, m: int):
+    """O5: keep the m candidates with the highest path confidence (product of the clamped
+    confidences from the root, float32), renumbered in candidate order.  parents / tokens
+    int32 [B, M], confidence float32 [B, M].  Returns dict(sel, parents, tokens, masks,
+    num_selected) with [B, m] arrays (-1 / 0 padded) and num_selected [B] (-1: bad tree)."""
+    par = np.ascontiguousarray(parents, np.int32)
+    tok = np.ascontiguousarray(tokens, np.int32)
+    conf = np.ascontiguousarray(confidence, np.float32)
+    B, M = par.shape
+    out = dict(sel=np.empty((B, m), np.int32), parents=np.empty((B, m), np.int32),
+               tokens=np.empty((B, m), np.int32), masks=np.empty((B, m), np.uint64),
+               num_selected=np.empty(B, np.int32))
+    lib().orc_tree_rerank(B, M, m, _p(par), _p(tok), _p(conf), _p(out["sel"]), _p(out["parents"]),
+                          _p(out["tokens"]), _p(out["masks"]), _p(out["num_selected"]))
+    return out

@@ -32,6 +32,13 @@
  *                        root-to-leaf order, are appended to the prefix K/V cache
  *                        and their hidden rows gathered, as sequential decoding of
  *                        those tokens would have left the cache.
+ *   O5 rerank           (EAGLE-2 blog, section 1: a draft token's confidence score
+ *                        approximates the probability that the target accepts it;
+ *                        section 4: after expansion, reranking keeps the tokens with
+ *                        the highest acceptance probability as the target's input):
+ *                        a node is reached only if its whole path is accepted, so its
+ *                        value is the product of the confidences along the path; the
+ *                        m highest-valued candidates form the verified tree.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - the adjusted distribution is norm(max(0, p - p_hat)) (standard speculative
@@ -521,6 +528,97 @@ void orc_commit(int B, int N, int Hkv, int D, int Lmax, int H, int esize,
         }
         new_lens[b] = L + n;
     }
+}
+
+/* ------------------------------------------------------------------ O5 rerank */
+
+typedef struct {
+    float value;
+    int32_t index;
+} orc_ranked;
+
+/* higher value first, then lower index */
+static int orc_rank_cmp(const void *a, const void *b)
+{
+    const orc_ranked *x = (const orc_ranked *)a, *y = (const orc_ranked *)b;
+    if (x->value > y->value) return -1;
+    if (x->value < y->value) return 1;
+    return (x->index > y->index) - (x->index < y->index);
+}
+
+static int orc_index_cmp(const void *a, const void *b)
+{
+    const int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+/* Reranking of an expanded candidate tree (M candidates, topological: parent[0] = -1,
+ * 0 <= parent[i] < i) down to the m-node tree the target verifies.
+ *   confidence c_i is clamped to [0, 1] (NaN and negatives count as 0; the root's is not used);
+ *   path value v_0 = 1, v_i = v_parent(i) * c_i in float32, root first (the decision is an
+ *     integer one, so both sides take it in the same precision: float32);
+ *   the k = min(m, M) candidates with the highest value are kept, ties to the lower index --
+ *     with c <= 1 a node's value never exceeds its parent's, so the kept set contains every
+ *     kept node's ancestors;
+ *   they are renumbered in increasing candidate index (a topological order, root = 0):
+ *     sel[t] = candidate index, parents_out[t] = new index of its parent, tokens_out[t],
+ *     masks_out[t] = bit j set for every kept ancestor-or-self j (k <= 64);
+ *   num_selected[b] = k, or -1 for a candidate tree that is not topological (nothing else
+ *     written for that sequence).
+ * Outputs are [B, m]; entries t >= k are -1 (masks 0). */
+void orc_tree_rerank(int B, int M, int m, const int32_t *parents, const int32_t *tokens,
+                     const float *confidence, int32_t *sel, int32_t *parents_out, int32_t *tokens_out,
+                     uint64_t *masks_out, int32_t *num_selected)
+{
+    orc_ranked *r = malloc(sizeof(orc_ranked) * (size_t)M);
+    float *v = malloc(sizeof(float) * (size_t)M);
+    int32_t *keep = malloc(sizeof(int32_t) * (size_t)M);
+    int32_t *newidx = malloc(sizeof(int32_t) * (size_t)M);
+    for (int b = 0; b < B; ++b) {
+        const int32_t *par = parents + (size_t)b * M;
+        const int32_t *tok = tokens + (size_t)b * M;
+        const float *c = confidence + (size_t)b * M;
+        int32_t *o_sel = sel + (size_t)b * m, *o_par = parents_out + (size_t)b * m;
+        int32_t *o_tok = tokens_out + (size_t)b * m;
+        uint64_t *o_mask = masks_out + (size_t)b * m;
+        for (int t = 0; t < m; ++t) {
+            o_sel[t] = o_par[t] = o_tok[t] = -1;
+            o_mask[t] = 0;
+        }
+        if (orc_check_tree(M, par) != ORC_OK) {
+            num_selected[b] = -1;
+            continue;
+        }
+        v[0] = 1.0f;
+        for (int i = 1; i < M; ++i) {
+            const float ci = c[i] > 0.0f ? (c[i] < 1.0f ? c[i] : 1.0f) : 0.0f;
+            v[i] = v[par[i]] * ci;
+        }
+        for (int i = 0; i < M; ++i) {
+            r[i].value = v[i];
+            r[i].index = i;
+        }
+        qsort(r, (size_t)M, sizeof(orc_ranked), orc_rank_cmp);
+        const int k = m < M ? m : M;
+        for (int t = 0; t < k; ++t) keep[t] = r[t].index;
+        qsort(keep, (size_t)k, sizeof(int32_t), orc_index_cmp);
+        for (int i = 0; i < M; ++i) newidx[i] = -1;
+        for (int t = 0; t < k; ++t) newidx[keep[t]] = t;
+        for (int t = 0; t < k; ++t) {
+            const int32_t i = keep[t];
+            o_sel[t] = i;
+            o_par[t] = i == 0 ? -1 : newidx[par[i]];
+            o_tok[t] = tok[i];
+            uint64_t mask = 0;
+            for (int32_t a = i; a >= 0; a = par[a]) mask |= 1ull << newidx[a];
+            o_mask[t] = mask;
+        }
+        num_selected[b] = k;
+    }
+    free(r);
+    free(v);
+    free(keep);
+    free(newidx);
 }
 
 /* Uniforms U(b, node, v, purpose) for v = 0..n-1 (test helper for the generator pins). */

@@ -585,7 +585,9 @@ void orc_tree_rerank(int B, int M, int m, const int32_t *parents, const int32_t 
             o_sel[t] = o_par[t] = o_tok[t] = -1;
             o_mask[t] = 0;
         }
-        if (orc_check_tree(M, par) != ORC_OK) {
+        int topo = M >= 1 && par[0] == -1;
+        for (int i = 1; topo && i < M; ++i) topo = par[i] >= 0 && par[i] < i;
+        if (!topo) {  /* candidate trees may exceed the 64 rows of a verified tree */
             num_selected[b] = -1;
             continue;
         }

@@ -50,8 +50,8 @@ def _check_structure(res, parents, tokens, b, m):
     return sel
 
 
-def test_chain_keeps_its_prefix(orc):
-    M, m = 20, 7
+@pytest.mark.parametrize("M,m", [(20, 7), (1024, 64)])
+def test_chain_keeps_its_prefix(orc, M, m):
     par = wl.chain_parents(M - 1)[None]
     rng = np.random.default_rng(1)
     conf = rng.uniform(0.05, 0.95, (1, M)).astype(np.float32)
@@ -61,9 +61,10 @@ def test_chain_keeps_its_prefix(orc):
     np.testing.assert_array_equal(_check_structure(res, par, tok, 0, m), np.arange(m))
 
 
-def test_equal_confidence_keeps_shallowest(orc):
+@pytest.mark.parametrize("M,m", [(40, 13), (300, 64)])
+def test_equal_confidence_keeps_shallowest(orc, M, m):
     rng = np.random.default_rng(2)
-    B, M, m = 4, 40, 13
+    B = 4
     par = np.stack([wl.random_parents(rng, M, 5) for _ in range(B)])
     tok = rng.integers(0, 1000, (B, M)).astype(np.int32)
     conf = np.full((B, M), 0.5, np.float32)
@@ -96,10 +97,10 @@ def test_star_keeps_most_confident_children(orc):
     np.testing.assert_array_equal(_check_structure(res, par, tok, 0, m), [0] + best)
 
 
-@pytest.mark.parametrize("seed", range(6))
-def test_kept_outvalue_dropped(orc, seed):
+@pytest.mark.parametrize("seed,M,m", [(s, 60, 20) for s in range(4)] + [(9, 500, 64), (10, 1024, 45)])
+def test_kept_outvalue_dropped(orc, seed, M, m):
     rng = np.random.default_rng(100 + seed)
-    B, M, m = 3, 60, 20
+    B = 3
     par = np.stack([wl.random_parents(rng, M, 6) for _ in range(B)])
     tok = rng.integers(0, 1000, (B, M)).astype(np.int32)
     conf = rng.uniform(0.02, 1.0, (B, M)).astype(np.float32)

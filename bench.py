@@ -32,6 +32,7 @@ import workloads as wl  # noqa: E402
 METRIC = "tree-verify steps/s and tree-tokens/s at 1 B200; achieved HBM GB/s as % of peak"
 L2_FLUSH_BYTES = 512 << 20
 FALLBACK_HBM_GBS = 6650.0
+RERANK_CANDIDATES = 256
 
 
 def _peaks():
@@ -304,6 +305,29 @@ def main():
     # each committed row: K and V of every kv head and one hidden row, read once, written once
     commit_bytes = commit_rows * (Hkv * D * el * 2 + H * el) * 2
 
+    # ---- EAGLE-2 reranking of an expanded candidate tree down to this workload's N nodes
+    # (timed on its own): RERANK_CANDIDATES candidates per sequence, random parents of depth
+    # <= 10 and uniform confidences, L2 flushed first
+    rr = np.random.default_rng(1234)
+    r_par = np.stack([wl.random_parents(rr, RERANK_CANDIDATES, 10) for _ in range(B)])
+    r_in = [torch.from_numpy(a).to(dev) for a in
+            (r_par.astype(np.int32), rr.integers(0, w.vocab, r_par.shape).astype(np.int32),
+             rr.uniform(0.0, 1.0, r_par.shape).astype(np.float32))]
+    r_out = [torch.empty((B, N), dtype=torch.int32, device=dev) for _ in range(3)]
+    r_masks = torch.empty((B, N), dtype=torch.int64, device=dev)
+    r_n = torch.empty((B,), dtype=torch.int32, device=dev)
+    rs_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    re_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        l2_flush()
+        rs_[i].record(stream)
+        binding.tree_rerank(*r_in, N, *r_out, r_masks, r_n)
+        re_[i].record(stream)
+    barrier()
+    rerank_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(rs_, re_)]))
+    assert (r_n.cpu().numpy() == min(N, RERANK_CANDIDATES)).all()
+
     # ---- end to end through the public API with host buffers: per-step tree inputs
     # (queries, tree K/V, hidden states, parents, tokens, draft distributions) copied from
     # pinned host memory, the walk's results read back; the prefix K/V cache and W stay
@@ -331,7 +355,8 @@ def main():
     assert binding.device_error(reset=True) == 0
 
     # ---- max over ranks
-    total_ms, e2e_ms, lm_ms, commit_ms = max_over_ranks([total_ms, e2e_ms, lm_ms, commit_ms], dist, dev)
+    total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms = max_over_ranks(
+        [total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms], dist, dev)
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -361,6 +386,8 @@ def main():
                    "rows": commit_rows, "bytes_per_launch": commit_bytes,
                    "achieved_gbs": commit_bytes / (commit_ms / 1e3) / 1e9,
                    "frac": commit_bytes / (commit_ms / 1e3) / 1e9 / peak, "bound": "latency"},
+        "rerank": {"kernel": "rerank_kernel", "us_per_launch": rerank_ms * 1e3,
+                   "candidates": RERANK_CANDIDATES, "kept": N, "bound": "latency"},
         "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "verify-steps/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -391,6 +418,11 @@ def main():
                           inp["parents"], acc_h, alen)
             reps += 1
         result["commit"]["oracle_us"] = (time.perf_counter() - t0) / reps * 1e6
+        t0, reps = time.perf_counter(), 0
+        while reps < 3 or time.perf_counter() - t0 < 1.0:
+            oracle.tree_rerank(r_par, r_in[1].cpu().numpy(), r_in[2].cpu().numpy(), N)
+            reps += 1
+        result["rerank"]["oracle_us"] = (time.perf_counter() - t0) / reps * 1e6
     print(json.dumps(result))
     if dist is not None:
         dist.destroy_process_group()

@@ -233,6 +233,36 @@ eagle_status_t eagle_commit_accepted(const eagle_shape_t *shape, void *k_prefix,
                                      void *feat, void *stream);
 
 /*
+ * EAGLE-2 reranking (EAGLE-2 blog, section 1: a draft token's confidence score
+ * approximates the probability that the target accepts it; section 4: after the expansion
+ * phase, reranking keeps the tokens with the highest acceptance probability as the target's
+ * input).  A candidate is reached only if its whole path is accepted, so per sequence b:
+ *     c_i = confidence clamped to [0, 1] (NaN and negatives count as 0; the root's is unused)
+ *     v_0 = 1,  v_i = v_parent(i) * c_i      float32, multiplied root first
+ * and the k = min(num_select, num_candidates) candidates with the highest v are kept, ties
+ * to the lower candidate index.  With c <= 1 no node outvalues its parent, so the kept set
+ * holds every kept node's ancestors; it is renumbered in increasing candidate index (a
+ * topological order, root = 0):
+ *     sel[b, t]          candidate index of kept node t
+ *     parents_out[b, t]  new index of its parent (-1 for the root)
+ *     tokens_out[b, t]   its token
+ *     masks_out[b, t]    bit j set for every kept ancestor-or-self j
+ *     num_selected[b]    k, or -1 if the candidate tree is not topological (parent[0] = -1,
+ *                        0 <= parent[i] < i)
+ * Entries t >= k are -1 (masks 0).  parents_out / tokens_out are the `parents` / `tokens` of
+ * the next eagle_verify_step (N = k); `sel` gathers its per-node rows from the candidates.
+ *   cand_parents, cand_tokens  [B, M] int32 device, confidence [B, M] float32 device
+ *   sel, parents_out, tokens_out [B, m] int32, masks_out [B, m] uint64 (8-byte aligned),
+ *   num_selected [B] int32
+ * 1 <= M (num_candidates) <= 1024, 1 <= m (num_select) <= 64, 1 <= B <= 65535; no workspace.
+ */
+eagle_status_t eagle_tree_rerank(int32_t batch, int32_t num_candidates, int32_t num_select,
+                                 const int32_t *cand_parents, const int32_t *cand_tokens,
+                                 const float *confidence, int32_t *sel, int32_t *parents_out,
+                                 int32_t *tokens_out, uint64_t *masks_out, int32_t *num_selected,
+                                 void *stream);
+
+/*
  * Reads (and, if `reset` != 0, clears) the device error word that bounded waits set
  * when they give up.  Synchronises the current device.  *code = 0 means no error.
  */

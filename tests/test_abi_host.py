@@ -143,6 +143,17 @@ def test_commit_checks_arguments_before_launch(lib):
     assert lib.eagle_commit_accepted(ctypes.byref(s_bad), *args, None) == binding.EAGLE_ERR_INVALID_ARGUMENT
 
 
+def test_rerank_checks_arguments_before_launch(lib):
+    p = [FAKE] * 8
+    ok = lambda B, M, m, masks=FAKE: lib.eagle_tree_rerank(B, M, m, *p[:6], masks, FAKE, None)
+    assert ok(1, 1025, 8) == binding.EAGLE_ERR_INVALID_ARGUMENT   # more candidates than a CTA
+    assert ok(1, 100, 65) == binding.EAGLE_ERR_INVALID_ARGUMENT   # more kept nodes than a mask
+    assert ok(1, 100, 0) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert ok(0, 100, 8) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert ok(1, 100, 8, masks=FAKE + 4) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert lib.eagle_tree_rerank(1, 100, 8, None, *p[:5], FAKE, FAKE, None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "nope.so"))
     monkeypatch.setattr(binding, "_lib", None)

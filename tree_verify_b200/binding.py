@@ -23,7 +23,7 @@ DTYPE_BF16 = 1
 
 EXPORTED = ("eagle_status_string", "eagle_workspace_bytes", "eagle_tree_attention",
             "eagle_lm_head_logits", "eagle_tree_accept", "eagle_verify_step",
-            "eagle_commit_accepted", "eagle_device_error")
+            "eagle_commit_accepted", "eagle_tree_rerank", "eagle_device_error")
 
 
 class Shape(ctypes.Structure):
@@ -77,6 +77,8 @@ def load() -> ctypes.CDLL:
     L.eagle_verify_step.argtypes = ([sp] + [vp] * 11 + [f32, u64, u64] + [vp] * 6 + [sz, vp])
     L.eagle_commit_accepted.restype = ctypes.c_int
     L.eagle_commit_accepted.argtypes = [sp] + [vp] * 12
+    L.eagle_tree_rerank.restype = ctypes.c_int
+    L.eagle_tree_rerank.argtypes = [i32, i32, i32] + [vp] * 9
     L.eagle_device_error.restype = ctypes.c_int
     L.eagle_device_error.argtypes = [ctypes.POINTER(i32), i32]
     _lib = L
@@ -162,6 +164,15 @@ def commit_accepted(shape: Shape, k_prefix, v_prefix, prefix_lens, k_tree, v_tre
         ctypes.byref(shape), _ptr(k_prefix), _ptr(v_prefix), _ptr(prefix_lens), _ptr(k_tree),
         _ptr(v_tree), _ptr(hidden), _ptr(parents), _ptr(accepted_nodes), _ptr(accept_len),
         _ptr(new_prefix_lens), _ptr(feat), _stream(stream)))
+
+
+def tree_rerank(cand_parents, cand_tokens, confidence, num_select: int, sel, parents_out,
+                tokens_out, masks_out, num_selected, stream=None) -> None:
+    B, M = cand_parents.shape
+    _check("eagle_tree_rerank", load().eagle_tree_rerank(
+        int(B), int(M), int(num_select), _ptr(cand_parents), _ptr(cand_tokens), _ptr(confidence),
+        _ptr(sel), _ptr(parents_out), _ptr(tokens_out), _ptr(masks_out), _ptr(num_selected),
+        _stream(stream)))
 
 
 def device_error(reset: bool = True) -> int:

@@ -16,6 +16,7 @@
 #include "attention.cuh"
 #include "attention_tc.cuh"
 #include "commit.cuh"
+#include "rerank.cuh"
 #include "device_common.cuh"
 #include "lm_head.cuh"
 
@@ -722,6 +723,24 @@ eagle_status_t eagle_commit_accepted(const eagle_shape_t* shape, void* k_prefix,
   if (rc != EAGLE_OK) return rc;
   return run_commit(shape, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, hidden, parents,
                     accepted_nodes, accept_len, new_prefix_lens, feat, static_cast<cudaStream_t>(stream));
+}
+
+eagle_status_t eagle_tree_rerank(int32_t batch, int32_t num_candidates, int32_t num_select,
+                                 const int32_t* cand_parents, const int32_t* cand_tokens,
+                                 const float* confidence, int32_t* sel, int32_t* parents_out,
+                                 int32_t* tokens_out, uint64_t* masks_out, int32_t* num_selected,
+                                 void* stream) {
+  if (batch < 1 || batch > 65535 || num_candidates < 1 || num_candidates > kRerankThreads ||
+      num_select < 1 || num_select > kRerankMaxSelect)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  if (cand_parents == nullptr || cand_tokens == nullptr || confidence == nullptr || sel == nullptr ||
+      parents_out == nullptr || tokens_out == nullptr || num_selected == nullptr ||
+      masks_out == nullptr || (reinterpret_cast<uintptr_t>(masks_out) & 7u) != 0)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  RerankParams p{cand_parents, cand_tokens, confidence, sel,        parents_out,
+                 tokens_out,   masks_out,   num_selected, num_candidates, num_select};
+  rerank_kernel<<<batch, kRerankThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
 }
 
 eagle_status_t eagle_device_error(int32_t* code, int32_t reset) {

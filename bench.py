@@ -269,6 +269,37 @@ def main():
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = float(np.sum(step_ms))
 
+    # ---- the same step replayed from a CUDA graph (one fixed seed/offset per capture),
+    # timed the same way: what launch gaps cost the stream-launched step
+    graph_info = {}
+    try:
+        gstream = torch.cuda.Stream(dev)
+        gstream.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gstream):
+            step.run(x, T, seed=rank, offset=0)  # warm the capture stream
+            gstream.synchronize()
+            with torch.cuda.graph(graph, stream=gstream):
+                step.run(x, T, seed=rank, offset=0, stream=gstream)
+        stream.wait_stream(gstream)
+        gs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ge = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            l2_flush()
+            gs[i].record(stream)
+            graph.replay()
+            ge[i].record(stream)
+        barrier()
+        graph_ms = float(np.mean([s_.elapsed_time(e_) for s_, e_ in zip(gs, ge)]))
+        assert binding.device_error(reset=True) == 0
+        graph_info = {"ms_per_step": graph_ms, "value": world / (graph_ms / 1e3),
+                      "note": "eagle_verify_step captured once (seed rank, offset 0) and replayed"}
+        del graph
+    except Exception as exc:  # capture is reported, never required
+        graph_info = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
+        torch.cuda.synchronize(dev)
+
     # ---- dominant kernel alone (LM head), same conditions, for the roofline
     ls = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     le = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -386,6 +417,7 @@ def main():
                    "rows": commit_rows, "bytes_per_launch": commit_bytes,
                    "achieved_gbs": commit_bytes / (commit_ms / 1e3) / 1e9,
                    "frac": commit_bytes / (commit_ms / 1e3) / 1e9 / peak, "bound": "latency"},
+        "graph": graph_info,
         "rerank": {"kernel": "rerank_kernel", "us_per_launch": rerank_ms * 1e3,
                    "candidates": RERANK_CANDIDATES, "kept": N, "bound": "latency"},
         "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "verify-steps/s",

@@ -15,6 +15,8 @@ Functions (each follows the passage cited in ``oracle.c``):
                         gather their hidden rows (EAGLE summary, section 3)
   tree_rerank     O5 -- the m candidates with the highest path confidence, renumbered as a
                         tree (EAGLE-2 blog, sections 1 and 4)
+  draft_select    O6 -- the children of draft nodes: top-k at T = 0, k races at T > 0
+                        (EAGLE summary, appendix A.1 "Tree Structure")
   race, uniform, philox -- the sampler and the counter-based generator it uses
 """
 from __future__ import annotations
@@ -62,6 +64,9 @@ def lib() -> ctypes.CDLL:
                                          ctypes.c_double, ctypes.c_int, vp, vp]
         L.orc_lm_head.argtypes = [ctypes.c_int] * 4 + [vp, vp, ctypes.c_int, vp, vp]
         L.orc_lm_head.restype = None
+        L.orc_draft_select.restype = None
+        L.orc_draft_select.argtypes = [ctypes.c_int] * 4 + [vp, ctypes.c_double, ctypes.c_uint64,
+                                       ctypes.c_uint64, ctypes.c_double, vp, vp, vp, vp]
         L.orc_tree_rerank.restype = None
         L.orc_tree_rerank.argtypes = [ctypes.c_int] * 3 + [vp] * 8
         L.orc_commit.restype = None
@@ -248,4 +253,21 @@ def tree_rerank(parents, tokens, confidence, m: int):
                num_selected=np.empty(B, np.int32))
     lib().orc_tree_rerank(B, M, m, _p(par), _p(tok), _p(conf), _p(out["sel"]), _p(out["parents"]),
                           _p(out["tokens"]), _p(out["masks"]), _p(out["num_selected"]))
+    return out
+
+
+def draft_select(logits, temperature: float, k: int, seed: int = 0, offset: int = 0,
+                 margin: float = 0.0, with_probs: bool = False):
+    """O6: children of draft nodes.  logits float32 [B, F, V]; returns dict(tokens [B, F, k]
+    int32, conf [B, F, k] float64, near [B, F, k] int32 and, if asked, probs [B, F, V])."""
+    lg = np.ascontiguousarray(logits, np.float32)
+    B, F, V = lg.shape
+    out = dict(tokens=np.empty((B, F, k), np.int32), conf=np.empty((B, F, k)),
+               near=np.empty((B, F, k), np.int32))
+    probs = np.empty((B, F, V)) if with_probs else None
+    lib().orc_draft_select(B, F, V, k, _p(lg), float(temperature), int(seed), int(offset),
+                           float(margin), _p(out["tokens"]), _p(out["conf"]), _p(probs),
+                           _p(out["near"]))
+    if with_probs:
+        out["probs"] = probs
     return out

@@ -286,17 +286,17 @@ void orc_lm_head(int M, int H, int V, int elem_type, const void *hidden, const v
 
 /* ------------------------------------------------------------------ O3 accept / resample */
 
-/* Exponential race: argmin over v with weight_v > 0 of (-ln U(b, node, v, 1)) / weight_v,
+/* Exponential race: argmin over v with weight_v > 0 of (-ln U(b, node, v, purpose)) / weight_v,
  * lowest v on ties.  *rel_gap receives (second - best) / best, or +inf if only one
  * candidate. */
-int32_t orc_race(int V, const double *weight, uint64_t seed, uint64_t offset, int32_t b,
-                 int32_t node, double *rel_gap)
+int32_t orc_race_purpose(int V, const double *weight, uint64_t seed, uint64_t offset, int32_t b,
+                         int32_t node, int32_t purpose, double *rel_gap)
 {
     double best = INFINITY, second = INFINITY;
     int32_t arg = -1;
     for (int v = 0; v < V; ++v) {
         if (!(weight[v] > 0.0)) continue;
-        const double e = -log(orc_uniform(seed, offset, b, node, v, 1));
+        const double e = -log(orc_uniform(seed, offset, b, node, v, purpose));
         const double key = e / weight[v];
         if (key < best) {
             second = best;
@@ -308,6 +308,13 @@ int32_t orc_race(int V, const double *weight, uint64_t seed, uint64_t offset, in
     }
     if (rel_gap) *rel_gap = (arg >= 0 && isfinite(second)) ? (second - best) / best : INFINITY;
     return arg;
+}
+
+/* The walk's sample (purpose 1). */
+int32_t orc_race(int V, const double *weight, uint64_t seed, uint64_t offset, int32_t b,
+                 int32_t node, double *rel_gap)
+{
+    return orc_race_purpose(V, weight, seed, offset, b, node, 1, rel_gap);
 }
 
 typedef struct {
@@ -621,6 +628,73 @@ void orc_tree_rerank(int B, int M, int m, const int32_t *parents, const int32_t 
     free(v);
     free(keep);
     free(newidx);
+}
+
+/* ------------------------------------------------------------------ O6 draft children */
+
+/* Children of the draft nodes (EAGLE summary, appendix A.1 "Tree Structure": in greedy
+ * decoding a node's children are the top k tokens by probability, in non-greedy decoding k
+ * tokens are sampled; section 3: the draft samples its next token through the LM head).
+ * Row (b, f) of logits [B, F, V] (float32) is draft node f of sequence b:
+ *   y = logit / T' with T' = T (T > 0) or 1 (T == 0); p = softmax(y) in float64;
+ *   T == 0: tokens = the k largest logits in decreasing order, ties to the lower index;
+ *   T  > 0: tokens[j] = the race over p with (node f, purpose 2 + j), j = 0..k-1: k
+ *           independent samples of p;
+ *   conf[j] = p[tokens[j]]; probs[v] = p_v when probs is not NULL;
+ *   near[j] = 1 when the decision is within `margin`: T == 0, the chosen logit and the next
+ *   one below it differ by at most margin * max(1, |logit|); T > 0, the race's best and
+ *   second keys are within margin (relative).
+ * Outputs are [B, F, k] (probs [B, F, V]). */
+void orc_draft_select(int B, int F, int V, int k, const float *logits, double T, uint64_t seed,
+                      uint64_t offset, double margin, int32_t *tokens, double *conf, double *probs,
+                      int32_t *near)
+{
+    double *p = malloc(sizeof(double) * (size_t)V);
+    const double Tp = T > 0.0 ? T : 1.0;
+    for (int b = 0; b < B; ++b) {
+        for (int f = 0; f < F; ++f) {
+            const size_t r = (size_t)b * F + f;
+            const float *l = logits + r * V;
+            double m = -INFINITY;
+            for (int v = 0; v < V; ++v) m = fmax(m, (double)l[v] / Tp);
+            double z = 0.0;
+            for (int v = 0; v < V; ++v) z += exp((double)l[v] / Tp - m);
+            for (int v = 0; v < V; ++v) p[v] = exp((double)l[v] / Tp - m) / z;
+            if (probs) memcpy(probs + r * V, p, sizeof(double) * (size_t)V);
+            int32_t *tok = tokens + r * k;
+            for (int j = 0; j < k; ++j) {
+                int32_t arg = -1;
+                int is_near = 0;
+                if (T > 0.0) {
+                    double gap;
+                    arg = orc_race_purpose(V, p, seed, offset, b, f, 2 + j, &gap);
+                    is_near = gap <= margin;
+                } else {
+                    /* the best logit not taken yet: strictly below the previous pick in
+                     * (value descending, index ascending) order */
+                    for (int v = 0; v < V; ++v) {
+                        if (j > 0) {
+                            const float pv = l[tok[j - 1]];
+                            if (!(l[v] < pv || (l[v] == pv && v > tok[j - 1]))) continue;
+                        }
+                        if (arg < 0 || l[v] > l[arg]) arg = v;
+                    }
+                    if (arg >= 0) {
+                        /* next value below the pick, for the margin */
+                        double nextv = -INFINITY;
+                        for (int v = 0; v < V; ++v)
+                            if (v != arg && (l[v] < l[arg] || (l[v] == l[arg] && v > arg)))
+                                nextv = fmax(nextv, l[v]);
+                        is_near = (double)l[arg] - nextv <= margin * fmax(1.0, fabs((double)l[arg]));
+                    }
+                }
+                tok[j] = arg;
+                conf[r * k + j] = arg >= 0 ? p[arg] : 0.0;
+                if (near) near[r * k + j] = is_near;
+            }
+        }
+    }
+    free(p);
 }
 
 /* Uniforms U(b, node, v, purpose) for v = 0..n-1 (test helper for the generator pins). */

@@ -33,6 +33,7 @@ METRIC = "tree-verify steps/s and tree-tokens/s at 1 B200; achieved HBM GB/s as 
 L2_FLUSH_BYTES = 512 << 20
 FALLBACK_HBM_GBS = 6650.0
 RERANK_CANDIDATES = 256
+DRAFT_ROWS, DRAFT_K = 10, 10
 
 
 def _peaks():
@@ -359,6 +360,26 @@ def main():
     rerank_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(rs_, re_)]))
     assert (r_n.cpu().numpy() == min(N, RERANK_CANDIDATES)).all()
 
+    # ---- children of DRAFT_ROWS draft nodes per sequence (DRAFT_K each) from draft LM-head
+    # logits over this vocabulary, at the step's temperature (timed on its own)
+    d_logits = torch.from_numpy((rr.standard_normal((B, DRAFT_ROWS, w.vocab)) * 2.0)
+                                .astype(np.float32)).to(dev)
+    d_tok = torch.empty((B, DRAFT_ROWS, DRAFT_K), dtype=torch.int32, device=dev)
+    d_conf = torch.empty((B, DRAFT_ROWS, DRAFT_K), dtype=torch.float32, device=dev)
+    d_probs = torch.empty_like(d_logits)
+    ds_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    de_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        l2_flush()
+        ds_[i].record(stream)
+        binding.draft_select(d_logits, T, DRAFT_K, rank, i, d_tok, d_conf, d_probs)
+        de_[i].record(stream)
+    barrier()
+    draft_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(ds_, de_)]))
+    assert binding.device_error(reset=True) == 0
+    draft_bytes = B * DRAFT_ROWS * w.vocab * 4 * 2  # logits read, distribution written
+
     # ---- end to end through the public API with host buffers: per-step tree inputs
     # (queries, tree K/V, hidden states, parents, tokens, draft distributions) copied from
     # pinned host memory, the walk's results read back; the prefix K/V cache and W stay
@@ -386,8 +407,8 @@ def main():
     assert binding.device_error(reset=True) == 0
 
     # ---- max over ranks
-    total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms = max_over_ranks(
-        [total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms], dist, dev)
+    total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms, draft_ms = max_over_ranks(
+        [total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms, draft_ms], dist, dev)
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -418,6 +439,12 @@ def main():
                    "achieved_gbs": commit_bytes / (commit_ms / 1e3) / 1e9,
                    "frac": commit_bytes / (commit_ms / 1e3) / 1e9 / peak, "bound": "latency"},
         "graph": graph_info,
+        "draft": {"kernel": "draft_select_kernel", "us_per_launch": draft_ms * 1e3,
+                  "rows": B * DRAFT_ROWS, "k": DRAFT_K, "vocab": w.vocab,
+                  "bytes_per_launch": draft_bytes,
+                  "achieved_gbs": draft_bytes / (draft_ms / 1e3) / 1e9,
+                  "frac": draft_bytes / (draft_ms / 1e3) / 1e9 / peak,
+                  "bound": "latency" if T == 0.0 else "alu (k Philox draws per entry)"},
         "rerank": {"kernel": "rerank_kernel", "us_per_launch": rerank_ms * 1e3,
                    "candidates": RERANK_CANDIDATES, "kept": N, "bound": "latency"},
         "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "verify-steps/s",
@@ -455,6 +482,12 @@ def main():
             oracle.tree_rerank(r_par, r_in[1].cpu().numpy(), r_in[2].cpu().numpy(), N)
             reps += 1
         result["rerank"]["oracle_us"] = (time.perf_counter() - t0) / reps * 1e6
+        lg_h = d_logits.cpu().numpy()
+        t0, reps = time.perf_counter(), 0
+        while reps < 1 or time.perf_counter() - t0 < 1.0:
+            oracle.draft_select(lg_h, T, DRAFT_K, seed=rank, offset=reps, with_probs=True)
+            reps += 1
+        result["draft"]["oracle_us"] = (time.perf_counter() - t0) / reps * 1e6
     print(json.dumps(result))
     if dist is not None:
         dist.destroy_process_group()

@@ -263,6 +263,31 @@ eagle_status_t eagle_tree_rerank(int32_t batch, int32_t num_candidates, int32_t 
                                  void *stream);
 
 /*
+ * Children of draft nodes (EAGLE summary, appendix A.1 "Tree Structure": in greedy decoding
+ * a node's children are the top k tokens by probability, in non-greedy decoding k tokens
+ * are sampled; section 3 "Drafting and verification": the draft samples its next token
+ * through the LM head).  Row (b, f) of `logits` is the draft LM head's output at draft node
+ * f of sequence b (eagle_lm_head_logits computes it):
+ *   T == 0: tokens[b, f, 0..k-1] = the k largest logits in decreasing order, ties to the
+ *           lower index (NaN is never chosen);
+ *   T  > 0: tokens[b, f, j] = argmin_v -ln U(b, f, v, 2 + j) / p_v, p = softmax(logits / T):
+ *           k independent samples of p (the exponential race with Philox purposes 2 .. k+1,
+ *           uniforms as for eagle_tree_accept);
+ *   conf[b, f, j] = the chosen token's probability (softmax(logits) at T == 0): the draft
+ *                   confidence eagle_tree_rerank takes;
+ *   probs[b, f, :] = p (softmax(logits) at T == 0) when probs is not NULL: the draft
+ *                   distribution eagle_tree_accept reads for the children drafted here.
+ * A row without a choosable token (all NaN) gives -1 and confidence 0.
+ *   logits  [B, F, V] float32 device;  tokens [B, F, k] int32;  conf [B, F, k] float32;
+ *   probs   [B, F, V] float32 or NULL
+ * 1 <= B <= 65535, 1 <= F (rows_per_seq) <= 256, 1 <= k <= 16, k <= V, T >= 0 finite.
+ */
+eagle_status_t eagle_draft_select(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
+                                  const float *logits, float temperature, uint64_t seed,
+                                  uint64_t offset, int32_t *tokens, float *conf, float *probs,
+                                  void *stream);
+
+/*
  * Reads (and, if `reset` != 0, clears) the device error word that bounded waits set
  * when they give up.  Synchronises the current device.  *code = 0 means no error.
  */

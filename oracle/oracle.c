@@ -673,6 +673,7 @@ void orc_draft_select(int B, int F, int V, int k, const float *logits, double T,
                     /* the best logit not taken yet: strictly below the previous pick in
                      * (value descending, index ascending) order */
                     for (int v = 0; v < V; ++v) {
+                        if (l[v] != l[v]) continue; /* NaN is never a child */
                         if (j > 0) {
                             const float pv = l[tok[j - 1]];
                             if (!(l[v] < pv || (l[v] == pv && v > tok[j - 1]))) continue;

@@ -154,6 +154,18 @@ def test_rerank_checks_arguments_before_launch(lib):
     assert lib.eagle_tree_rerank(1, 100, 8, None, *p[:5], FAKE, FAKE, None) == binding.EAGLE_ERR_INVALID_ARGUMENT
 
 
+def test_draft_select_checks_arguments_before_launch(lib):
+    call = lambda B, F, V, k, T=1.0, lg=FAKE: lib.eagle_draft_select(B, F, V, k, lg, T, 0, 0, FAKE,
+                                                                     FAKE, None, None)
+    assert call(1, 4, 1000, 17) == binding.EAGLE_ERR_INVALID_ARGUMENT   # more than 16 children
+    assert call(1, 4, 8, 10) == binding.EAGLE_ERR_INVALID_ARGUMENT      # k > V
+    assert call(1, 257, 1000, 4) == binding.EAGLE_ERR_INVALID_ARGUMENT  # node field is 8 bits
+    assert call(0, 4, 1000, 4) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 1000, 4, T=-1.0) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 1000, 4, T=float("nan")) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 1000, 4, lg=None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "nope.so"))
     monkeypatch.setattr(binding, "_lib", None)

@@ -23,7 +23,8 @@ DTYPE_BF16 = 1
 
 EXPORTED = ("eagle_status_string", "eagle_workspace_bytes", "eagle_tree_attention",
             "eagle_lm_head_logits", "eagle_tree_accept", "eagle_verify_step",
-            "eagle_commit_accepted", "eagle_tree_rerank", "eagle_device_error")
+            "eagle_commit_accepted", "eagle_tree_rerank", "eagle_draft_select",
+            "eagle_device_error")
 
 
 class Shape(ctypes.Structure):
@@ -79,6 +80,8 @@ def load() -> ctypes.CDLL:
     L.eagle_commit_accepted.argtypes = [sp] + [vp] * 12
     L.eagle_tree_rerank.restype = ctypes.c_int
     L.eagle_tree_rerank.argtypes = [i32, i32, i32] + [vp] * 9
+    L.eagle_draft_select.restype = ctypes.c_int
+    L.eagle_draft_select.argtypes = [i32, i32, i32, i32, vp, f32, u64, u64, vp, vp, vp, vp]
     L.eagle_device_error.restype = ctypes.c_int
     L.eagle_device_error.argtypes = [ctypes.POINTER(i32), i32]
     _lib = L
@@ -173,6 +176,14 @@ def tree_rerank(cand_parents, cand_tokens, confidence, num_select: int, sel, par
         int(B), int(M), int(num_select), _ptr(cand_parents), _ptr(cand_tokens), _ptr(confidence),
         _ptr(sel), _ptr(parents_out), _ptr(tokens_out), _ptr(masks_out), _ptr(num_selected),
         _stream(stream)))
+
+
+def draft_select(logits, temperature: float, k: int, seed: int, offset: int, tokens, conf,
+                 probs=None, stream=None) -> None:
+    B, F, V = logits.shape
+    _check("eagle_draft_select", load().eagle_draft_select(
+        int(B), int(F), int(V), int(k), _ptr(logits), float(temperature), int(seed), int(offset),
+        _ptr(tokens), _ptr(conf), _ptr(probs), _stream(stream)))
 
 
 def device_error(reset: bool = True) -> int:

@@ -16,6 +16,7 @@
 #include "attention.cuh"
 #include "attention_tc.cuh"
 #include "commit.cuh"
+#include "draft.cuh"
 #include "rerank.cuh"
 #include "device_common.cuh"
 #include "lm_head.cuh"
@@ -740,6 +741,25 @@ eagle_status_t eagle_tree_rerank(int32_t batch, int32_t num_candidates, int32_t 
   RerankParams p{cand_parents, cand_tokens, confidence, sel,        parents_out,
                  tokens_out,   masks_out,   num_selected, num_candidates, num_select};
   rerank_kernel<<<batch, kRerankThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
+}
+
+eagle_status_t eagle_draft_select(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
+                                  const float* logits, float temperature, uint64_t seed,
+                                  uint64_t offset, int32_t* tokens, float* conf, float* probs,
+                                  void* stream) {
+  if (batch < 1 || batch > 65535 || rows_per_seq < 1 || rows_per_seq > 256 || k < 1 ||
+      k > kDraftMaxK || vocab < k)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  if (!(temperature >= 0.f) || !std::isfinite(temperature)) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (logits == nullptr || tokens == nullptr || conf == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
+  DraftParams p{logits, tokens, conf, probs, rows_per_seq, vocab, k, temperature, seed, offset};
+  const long rows = static_cast<long>(batch) * rows_per_seq;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (temperature == 0.f)
+    draft_select_kernel<true><<<static_cast<unsigned>(rows), kDraftThreads, 0, st>>>(p);
+  else
+    draft_select_kernel<false><<<static_cast<unsigned>(rows), kDraftThreads, 0, st>>>(p);
   return launch_status();
 }
 

@@ -52,15 +52,20 @@ struct AccParams {
 };
 
 // ---------------------------------------------------------------- reduction operators
-// Payload float4.  Every operator is commutative, so a butterfly leaves all lanes equal.
-// Components .z/.w of OpMaxSum and .y/.z/.w of OpSum are "owner fields": exactly one CTA
-// contributes a nonzero value (a scalar it alone holds in shared memory) and the others
-// contribute 0, so adding them broadcasts that scalar exactly.
+// Payload float4.  Every operator is commutative bit for bit, so a butterfly leaves all
+// lanes equal.  Components .z/.w of OpMaxSum and .y/.z/.w of OpSum are "owner fields":
+// exactly one CTA contributes a nonzero value (a scalar it alone holds in shared memory)
+// and the others contribute 0, so adding them broadcasts that scalar exactly.
 struct OpMaxSum {  // (max y, sum exp(y - max), owner fields)
   static __device__ __forceinline__ float4 identity() { return make_float4(-INFINITY, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ float4 operator()(float4 a, float4 b) const {
     const float m = fmaxf(a.x, b.x);
-    const float s = m == -INFINITY ? 0.f : a.y * __expf(a.x - m) + b.y * __expf(b.x - m);
+    // each product rounded on its own: a contracted a*x + b*y (one product fused into the
+    // add) rounds differently from b*y + a*x, and lanes holding op(a, b) and op(b, a)
+    // would then disagree on Z
+    const float s = m == -INFINITY
+                        ? 0.f
+                        : __fadd_rn(__fmul_rn(a.y, __expf(a.x - m)), __fmul_rn(b.y, __expf(b.x - m)));
     return make_float4(m, s, a.z + b.z, a.w + b.w);
   }
 };

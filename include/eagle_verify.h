@@ -280,7 +280,10 @@ eagle_status_t eagle_tree_rerank(int32_t batch, int32_t num_candidates, int32_t 
  * A row without a choosable token (all NaN) gives -1 and confidence 0.
  *   logits  [B, F, V] float32 device;  tokens [B, F, k] int32;  conf [B, F, k] float32;
  *   probs   [B, F, V] float32 or NULL
- * 1 <= B <= 65535, 1 <= F (rows_per_seq) <= 256, 1 <= k <= 16, k <= V, T >= 0 finite.
+ * 1 <= B <= 65535, 1 <= F (rows_per_seq) <= 256, 1 <= k <= 16, k <= V, T >= 0 finite,
+ * logits 4-byte aligned (else EAGLE_ERR_INVALID_ARGUMENT).  A row is split over a cluster of
+ * up to 8 CTAs, each holding its slice in shared memory, so V <= 393216 (else
+ * EAGLE_ERR_UNSUPPORTED).  No workspace.
  */
 eagle_status_t eagle_draft_select(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
                                   const float *logits, float temperature, uint64_t seed,

@@ -164,6 +164,9 @@ def test_draft_select_checks_arguments_before_launch(lib):
     assert call(1, 4, 1000, 4, T=-1.0) == binding.EAGLE_ERR_INVALID_ARGUMENT
     assert call(1, 4, 1000, 4, T=float("nan")) == binding.EAGLE_ERR_INVALID_ARGUMENT
     assert call(1, 4, 1000, 4, lg=None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 1000, 4, lg=FAKE + 2) == binding.EAGLE_ERR_INVALID_ARGUMENT  # not a float address
+    # a row is staged in the shared memory of at most 8 CTAs (192 KB each)
+    assert call(1, 4, 8 * 49152 + 1, 4) == binding.EAGLE_ERR_UNSUPPORTED
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

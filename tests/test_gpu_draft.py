@@ -1,7 +1,8 @@
 """eagle_draft_select on the GPU against oracle O6: greedy children bit for bit (ties to
 the lower index included), sampled children wherever the oracle's race is not a near tie
 (margin 1e-4, as for the walk), confidences and row distributions within 1e-5 relative;
-vocabularies with a ragged tail and the 128256-token vocabulary, k from 1 to 16."""
+vocabularies with a ragged tail and the 128256-token vocabulary, k from 1 to 16, rows on
+one CTA and rows split over a cluster."""
 import numpy as np
 import pytest
 import torch
@@ -23,7 +24,10 @@ def _run(cuda_lib, logits, T, k, seed, offset, with_probs=True):
     return tok.cpu().numpy(), conf.cpu().numpy(), None if probs is None else probs.cpu().numpy()
 
 
-CASES = [(2, 3, 1000, 4), (1, 8, 32000, 10), (3, 2, 1001, 16), (1, 2, 128256, 8), (4, 5, 777, 1)]
+# rows of one CTA (small vocabularies, many rows) and rows split over clusters of 2 to 8 CTAs
+# (large vocabularies, few rows), with ragged last slices (8195 = 7 * 1028 + 999)
+CASES = [(2, 3, 1000, 4), (1, 8, 32000, 10), (3, 2, 1001, 16), (1, 2, 128256, 8), (4, 5, 777, 1),
+         (1, 3, 8195, 5), (4, 8, 32000, 4), (2, 100, 4096, 3)]
 
 
 @pytest.mark.parametrize("T", [0.0, 0.7, 1.0])

@@ -244,6 +244,13 @@ struct DeviceState {
   cudaEvent_t lm_mark = nullptr;  // LM head under way (T = 0 beside it) or completed
   cudaEvent_t attn_done = nullptr;
   std::mutex step_mu;  // one step's fork/join sequence at a time on the shared side stream
+  // eagle_draft_select: shared-memory limits set once; clusters of S CTAs resident at once,
+  // [greedy][log2 S][slice bytes in 4 KB steps], stored + 1 (0: not queried yet)
+  std::once_flag draft_once;
+  bool draft_ok = false;
+  int draft_max_cluster = kDraftPortableCluster;  // 16 where the device co-schedules them
+  std::mutex draft_mu;
+  int draft_clusters[2][5][kDraftMaxSmem / 4096 + 1] = {};
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -590,6 +597,81 @@ bool device_accept_supported(const eagle_shape_t* s, int dev) {
   return ap.nq >= 1 && ap.smem <= kAccMaxSmem;
 }
 
+template <bool kGreedy>
+int draft_active_clusters(int S, size_t smem) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(S));
+  cfg.blockDim = dim3(kDraftThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, draft_select_kernel<kGreedy>, &cfg) != cudaSuccess) n = 0;
+  cudaGetLastError();
+  return n;
+}
+
+// Entries per CTA when a row of V entries is split over S CTAs (a multiple of 4).
+int draft_slice(int V, int S) { return (((V + S - 1) / S + 3) / 4) * 4; }
+
+// Cluster size for `rows` rows of V entries, each CTA staging its slice in shared memory:
+// the largest S in {16, 8, 4, 2} whose clusters are all resident at once, with slices of at
+// least 1024 entries; else the smallest S whose slice fits (more rows than one wave holds
+// gain nothing from splitting).  0: no S fits.
+int draft_cluster(int dev, long rows, int V, bool greedy) {
+  DeviceState& ds = g_dev[dev];
+  int first_fit = 0;
+  for (int lg = 0; lg < 4; ++lg) {  // portable sizes only
+    const int S = 1 << lg;
+    if (static_cast<size_t>(draft_slice(V, S)) * 4 <= kDraftMaxSmem) {
+      first_fit = S;
+      break;
+    }
+  }
+  if (first_fit == 0) return 0;
+  for (int lg = 4; lg >= 1; --lg) {
+    const int S = 1 << lg;
+    const size_t bytes = static_cast<size_t>(draft_slice(V, S)) * 4;
+    if (S > ds.draft_max_cluster || S < first_fit || V < S * 1024 || bytes > kDraftMaxSmem) continue;
+    const size_t bucket = (bytes + 4095) / 4096;
+    int n;
+    {
+      std::lock_guard<std::mutex> lock(ds.draft_mu);
+      int& slot = ds.draft_clusters[greedy ? 1 : 0][lg][bucket];
+      if (slot == 0)
+        slot = 1 + (greedy ? draft_active_clusters<true>(S, bucket * 4096)
+                           : draft_active_clusters<false>(S, bucket * 4096));
+      n = slot - 1;
+    }
+    if (rows <= n) return S;
+  }
+  return first_fit;
+}
+
+bool ensure_draft(int dev) {
+  DeviceState& ds = g_dev[dev];
+  std::call_once(ds.draft_once, [&] {
+    const int bytes = static_cast<int>(kDraftMaxSmem);
+    ds.draft_ok = cudaFuncSetAttribute(draft_select_kernel<true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+                  cudaFuncSetAttribute(draft_select_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+    if (cudaFuncSetAttribute(draft_select_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(draft_select_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess &&
+        draft_active_clusters<true>(16, 4096) >= 1 && draft_active_clusters<false>(16, 4096) >= 1)
+      ds.draft_max_cluster = 16;
+    cudaGetLastError();
+  });
+  return ds.draft_ok;
+}
+
 }  // namespace
 }  // namespace eagle
 
@@ -753,13 +835,33 @@ eagle_status_t eagle_draft_select(int32_t batch, int32_t rows_per_seq, int32_t v
     return EAGLE_ERR_INVALID_ARGUMENT;
   if (!(temperature >= 0.f) || !std::isfinite(temperature)) return EAGLE_ERR_INVALID_ARGUMENT;
   if (logits == nullptr || tokens == nullptr || conf == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
-  DraftParams p{logits, tokens, conf, probs, rows_per_seq, vocab, k, temperature, seed, offset};
+  if ((reinterpret_cast<uintptr_t>(logits) & 3) != 0) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (static_cast<size_t>(draft_slice(vocab, kDraftPortableCluster)) * 4 > kDraftMaxSmem)
+    return EAGLE_ERR_UNSUPPORTED;  // a row must fit the shared memory of one cluster
+  int dev;
+  if (!current_device(&dev) || !ensure_draft(dev)) return EAGLE_ERR_CUDA;
   const long rows = static_cast<long>(batch) * rows_per_seq;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (temperature == 0.f)
-    draft_select_kernel<true><<<static_cast<unsigned>(rows), kDraftThreads, 0, st>>>(p);
-  else
-    draft_select_kernel<false><<<static_cast<unsigned>(rows), kDraftThreads, 0, st>>>(p);
+  const bool greedy = temperature == 0.f;
+  const int S = draft_cluster(dev, rows, vocab, greedy);
+  if (S == 0) return EAGLE_ERR_UNSUPPORTED;
+  const int slice = draft_slice(vocab, S);
+  const int vec16 = (vocab % 4 == 0 && aligned16(logits)) ? 1 : 0;
+  DraftParams p{logits, tokens, conf, probs, rows_per_seq, vocab, k, slice, vec16, temperature, seed, offset};
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * S));
+  cfg.blockDim = dim3(kDraftThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(slice) * 4;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = greedy ? cudaLaunchKernelEx(&cfg, draft_select_kernel<true>, p)
+                               : cudaLaunchKernelEx(&cfg, draft_select_kernel<false>, p);
+  if (e != cudaSuccess) return EAGLE_ERR_CUDA;
   return launch_status();
 }
 

@@ -17,6 +17,8 @@ Functions (each follows the passage cited in ``oracle.c``):
                         tree (EAGLE-2 blog, sections 1 and 4)
   draft_select    O6 -- the children of draft nodes: top-k at T = 0, k races at T > 0
                         (EAGLE summary, appendix A.1 "Tree Structure")
+  draft_select_distinct, draft_child_rows
+                  O7 -- siblings drawn without replacement and the row each was drawn from
   race, uniform, philox -- the sampler and the counter-based generator it uses
 """
 from __future__ import annotations
@@ -65,6 +67,11 @@ def lib() -> ctypes.CDLL:
         L.orc_lm_head.argtypes = [ctypes.c_int] * 4 + [vp, vp, ctypes.c_int, vp, vp]
         L.orc_lm_head.restype = None
         L.orc_draft_select.restype = None
+        L.orc_draft_select_distinct.restype = None
+        L.orc_draft_select_distinct.argtypes = [ctypes.c_int] * 4 + [vp, ctypes.c_double, ctypes.c_uint64,
+                                                 ctypes.c_uint64, ctypes.c_double, vp, vp, vp, vp]
+        L.orc_draft_child_rows.restype = None
+        L.orc_draft_child_rows.argtypes = [ctypes.c_int] * 4 + [vp, vp, vp]
         L.orc_draft_select.argtypes = [ctypes.c_int] * 4 + [vp, ctypes.c_double, ctypes.c_uint64,
                                        ctypes.c_uint64, ctypes.c_double, vp, vp, vp, vp]
         L.orc_tree_rerank.restype = None
@@ -270,4 +277,33 @@ def draft_select(logits, temperature: float, k: int, seed: int = 0, offset: int 
                            _p(out["near"]))
     if with_probs:
         out["probs"] = probs
+    return out
+
+
+def draft_select_distinct(logits, temperature: float, k: int, seed: int = 0, offset: int = 0,
+                          margin: float = 0.0, with_probs: bool = False):
+    """O7: k siblings drawn without replacement (the k smallest clocks of one race, purpose 2;
+    the top k logits at T = 0).  Same arguments and outputs as draft_select."""
+    lg = np.ascontiguousarray(logits, np.float32)
+    B, F, V = lg.shape
+    out = dict(tokens=np.empty((B, F, k), np.int32), conf=np.empty((B, F, k)),
+               near=np.empty((B, F, k), np.int32))
+    probs = np.empty((B, F, V)) if with_probs else None
+    lib().orc_draft_select_distinct(B, F, V, k, _p(lg), float(temperature), int(seed), int(offset),
+                                    float(margin), _p(out["tokens"]), _p(out["conf"]), _p(probs),
+                                    _p(out["near"]))
+    if with_probs:
+        out["probs"] = probs
+    return out
+
+
+def draft_child_rows(probs, tokens):
+    """O7: the row each sibling was drawn from: probs [B, F, V], tokens [B, F, k] ->
+    [B, F, k, V] float64, row j = probs without tokens[..., :j], renormalised."""
+    pr = np.ascontiguousarray(probs, np.float64)
+    tk = np.ascontiguousarray(tokens, np.int32)
+    B, F, V = pr.shape
+    k = tk.shape[-1]
+    out = np.empty((B, F, k, V))
+    lib().orc_draft_child_rows(B, F, V, k, _p(pr), _p(tk), _p(out))
     return out

@@ -698,6 +698,100 @@ void orc_draft_select(int B, int F, int V, int k, const float *logits, double T,
     free(p);
 }
 
+/* O7: siblings drawn without replacement (EAGLE summary, appendix A.1 "Tree Structure": k
+ * tokens are sampled for a node's children; sampling them without replacement keeps the
+ * siblings distinct).  Row (b, f) as in O6, p = softmax(logits / T') in float64:
+ *   T == 0: the k largest logits (as O6: distinct by construction);
+ *   T  > 0: the k smallest clocks E_v / p_v, E_v = -ln U(b, f, v, purpose 2), in increasing
+ *           order, over the tokens with p_v > 0 (fewer than k such tokens: -1 after them).
+ *           The clocks of independent exponentials come out in the order of successive draws
+ *           without replacement: the first is a draw from p, each later one a draw from p
+ *           restricted to the tokens not drawn yet.
+ *   conf[j] = p[tokens[j]]; probs = p when not NULL;
+ *   near[j] = 1 when clock j is within `margin` (relative) of clock j + 1 or of clock j - 1
+ *   (T == 0: O6's rule). */
+static int orc_cmp_clock(const void *a, const void *b)
+{
+    const double *x = (const double *)a, *y = (const double *)b;
+    if (x[0] < y[0]) return -1;
+    if (x[0] > y[0]) return 1;
+    return x[1] < y[1] ? -1 : (x[1] > y[1] ? 1 : 0);
+}
+
+void orc_draft_select_distinct(int B, int F, int V, int k, const float *logits, double T,
+                               uint64_t seed, uint64_t offset, double margin, int32_t *tokens,
+                               double *conf, double *probs, int32_t *near)
+{
+    if (!(T > 0.0)) {
+        orc_draft_select(B, F, V, k, logits, T, seed, offset, margin, tokens, conf, probs, near);
+        return;
+    }
+    double *p = malloc(sizeof(double) * (size_t)V);
+    double *clk = malloc(sizeof(double) * 2 * (size_t)V); /* (clock, token) pairs */
+    for (int b = 0; b < B; ++b) {
+        for (int f = 0; f < F; ++f) {
+            const size_t r = (size_t)b * F + f;
+            const float *l = logits + r * V;
+            double m = -INFINITY;
+            for (int v = 0; v < V; ++v) m = fmax(m, (double)l[v] / T);
+            double z = 0.0;
+            for (int v = 0; v < V; ++v) z += exp((double)l[v] / T - m);
+            for (int v = 0; v < V; ++v) p[v] = exp((double)l[v] / T - m) / z;
+            if (probs) memcpy(probs + r * V, p, sizeof(double) * (size_t)V);
+            int n = 0;
+            for (int v = 0; v < V; ++v) {
+                if (!(p[v] > 0.0)) continue;
+                clk[2 * n] = -log(orc_uniform(seed, offset, b, f, v, 2)) / p[v];
+                clk[2 * n + 1] = v;
+                ++n;
+            }
+            qsort(clk, (size_t)n, 2 * sizeof(double), orc_cmp_clock);
+            for (int j = 0; j < k; ++j) {
+                const int have = j < n;
+                tokens[r * k + j] = have ? (int32_t)clk[2 * j + 1] : -1;
+                conf[r * k + j] = have ? p[(int)clk[2 * j + 1]] : 0.0;
+                if (near) {
+                    int is_near = 0;
+                    if (have && j + 1 < n) is_near |= (clk[2 * j + 2] - clk[2 * j]) <= margin * clk[2 * j];
+                    if (have && j > 0) is_near |= (clk[2 * j] - clk[2 * j - 2]) <= margin * clk[2 * j - 2];
+                    near[r * k + j] = is_near;
+                }
+            }
+        }
+    }
+    free(clk);
+    free(p);
+}
+
+/* O7: the row each sibling was drawn from.  Child j of row (b, f) was drawn from p with the
+ * earlier siblings' tokens removed, so its row is
+ *   q_j(v) = p_v / R_j for v not in {t_0 .. t_{j-1}}, 0 otherwise,  R_j = the sum of p over
+ *   the tokens not removed (summed directly, not as 1 minus the removed mass);
+ * q_0 = p, and a row with R_j = 0 (or a token -1 before it) is all zeros.  probs [B, F, V],
+ * tokens [B, F, k] -> child [B, F, k, V], float64. */
+void orc_draft_child_rows(int B, int F, int V, int k, const double *probs, const int32_t *tokens,
+                          double *child)
+{
+    unsigned char *gone = malloc((size_t)V);
+    for (size_t r = 0; r < (size_t)B * F; ++r) {
+        const double *p = probs + r * V;
+        memset(gone, 0, (size_t)V);
+        int dead = 0;
+        for (int j = 0; j < k; ++j) {
+            double *q = child + (r * k + j) * V;
+            double R = 0.0;
+            if (!dead)
+                for (int v = 0; v < V; ++v)
+                    if (!gone[v]) R += p[v];
+            for (int v = 0; v < V; ++v) q[v] = (!dead && !gone[v] && R > 0.0) ? p[v] / R : 0.0;
+            const int32_t t = tokens[r * k + j];
+            if (t < 0 || t >= V) dead = 1;
+            else gone[t] = 1;
+        }
+    }
+    free(gone);
+}
+
 /* Uniforms U(b, node, v, purpose) for v = 0..n-1 (test helper for the generator pins). */
 void orc_fill_uniforms(uint64_t seed, uint64_t offset, int32_t b, int32_t node, int32_t purpose,
                        int32_t n, double *out)

@@ -34,6 +34,7 @@ L2_FLUSH_BYTES = 512 << 20
 FALLBACK_HBM_GBS = 6650.0
 RERANK_CANDIDATES = 256
 DRAFT_ROWS, DRAFT_K = 10, 10
+STACK_LAYERS = 32  # the stacked-attention workload: one verify pass through every layer
 
 
 def _peaks():
@@ -380,6 +381,58 @@ def main():
     assert binding.device_error(reset=True) == 0
     draft_bytes = B * DRAFT_ROWS * w.vocab * 4 * 2  # logits read, distribution written
 
+    # ---- the same children drawn without replacement, then the row each was drawn from
+    # (timed together and the rows alone, each L2-flushed)
+    d_rows = torch.empty((B, DRAFT_ROWS, DRAFT_K, w.vocab), dtype=torch.float32, device=dev)
+    dd_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dd_m = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dd_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        l2_flush()
+        dd_s[i].record(stream)
+        binding.draft_select_distinct(d_logits, T, DRAFT_K, rank, i, d_tok, d_conf, d_probs)
+        dd_m[i].record(stream)
+        binding.draft_child_rows(d_probs, d_tok, d_rows)
+        dd_e[i].record(stream)
+    barrier()
+    distinct_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(dd_s, dd_m)]))
+    rows_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(dd_m, dd_e)]))
+    assert binding.device_error(reset=True) == 0
+    rows_bytes = B * DRAFT_ROWS * w.vocab * 4 * (1 + DRAFT_K)  # distribution read, k rows written
+
+    # ---- stacked layers: the tree attention of every layer of a STACK_LAYERS-layer model,
+    # each layer with its own prefix K/V cache, queries and tree K/V (seeded device normals),
+    # back to back as in one verify pass; the caches (STACK_LAYERS x the step's) exceed L2
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321 + rank)
+    kv_dt = x.k_prefix.dtype
+    def _layers(t):
+        return torch.randn((STACK_LAYERS,) + tuple(t.shape), generator=gen, device=dev,
+                           dtype=torch.float32).to(kv_dt)
+    st_q, st_kp, st_vp, st_kt, st_vt = (_layers(t) for t in (x.q, x.k_prefix, x.v_prefix, x.k_tree, x.v_tree))
+    st_out = torch.empty_like(st_q)
+    def stacked_pass():
+        for l in range(STACK_LAYERS):
+            binding.tree_attention(step.shape, st_q[l], st_kp[l], st_vp[l], x.prefix_lens, st_kt[l], st_vt[l],
+                                   x.parents, st_out[l], step.workspace, stream)
+    stacked_pass()
+    torch.cuda.synchronize(dev)
+    ss_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    se_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        l2_flush()
+        ss_[i].record(stream)
+        stacked_pass()
+        se_[i].record(stream)
+    barrier()
+    stacked_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(ss_, se_)]))
+    assert binding.device_error(reset=True) == 0
+    lens_h = x.prefix_lens.cpu().numpy().astype(np.int64)
+    stacked_kv = int(STACK_LAYERS * lens_h.sum() * w.num_kv_heads * w.head_dim * 2 * x.k_prefix.element_size())
+    del st_q, st_kp, st_vp, st_kt, st_vt, st_out
+
     # ---- end to end through the public API with host buffers: per-step tree inputs
     # (queries, tree K/V, hidden states, parents, tokens, draft distributions) copied from
     # pinned host memory, the walk's results read back; the prefix K/V cache and W stay
@@ -407,8 +460,8 @@ def main():
     assert binding.device_error(reset=True) == 0
 
     # ---- max over ranks
-    total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms, draft_ms = max_over_ranks(
-        [total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms, draft_ms], dist, dev)
+    total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms, draft_ms, distinct_ms, rows_ms, stacked_ms = max_over_ranks(
+        [total_ms, e2e_ms, lm_ms, commit_ms, rerank_ms, draft_ms, distinct_ms, rows_ms, stacked_ms], dist, dev)
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -445,6 +498,17 @@ def main():
                   "achieved_gbs": draft_bytes / (draft_ms / 1e3) / 1e9,
                   "frac": draft_bytes / (draft_ms / 1e3) / 1e9 / peak,
                   "bound": "latency" if T == 0.0 else "alu (k Philox draws per entry)"},
+        "draft_distinct": {"kernel": "draft_select_kernel (one race) + draft_child_rows_kernel",
+                           "select_us": distinct_ms * 1e3, "child_rows_us": rows_ms * 1e3,
+                           "child_rows_bytes": rows_bytes,
+                           "child_rows_frac": rows_bytes / (rows_ms / 1e3) / 1e9 / peak},
+        "stacked_layers": {"workload": f"{w.name}, tree attention of {STACK_LAYERS} layers per pass, "
+                                       "own caches per layer",
+                           "layers": STACK_LAYERS, "us_per_pass": stacked_ms * 1e3,
+                           "us_per_layer": stacked_ms * 1e3 / STACK_LAYERS,
+                           "prefix_kv_bytes_per_pass": stacked_kv,
+                           "achieved_gbs": stacked_kv / (stacked_ms / 1e3) / 1e9,
+                           "frac": stacked_kv / (stacked_ms / 1e3) / 1e9 / peak},
         "rerank": {"kernel": "rerank_kernel", "us_per_launch": rerank_ms * 1e3,
                    "candidates": RERANK_CANDIDATES, "kept": N, "bound": "latency"},
         "e2e": {"value": world * args.steps / (e2e_ms / 1e3), "unit": "verify-steps/s",

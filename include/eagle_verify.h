@@ -291,6 +291,40 @@ eagle_status_t eagle_draft_select(int32_t batch, int32_t rows_per_seq, int32_t v
                                   void *stream);
 
 /*
+ * Children of draft nodes drawn WITHOUT replacement (EAGLE summary, appendix A.1 "Tree
+ * Structure": k tokens are sampled for a node's children; drawn without replacement they
+ * are distinct).  Same arguments, layouts, limits and outputs as eagle_draft_select, except:
+ *   T > 0: tokens[b, f, 0..k-1] = the k smallest keys -ln U(b, f, v, 2) / p_v of ONE
+ *          exponential race (Philox purpose 2), in increasing order: successive draws
+ *          without replacement from p (the first is a draw from p, each later one a draw
+ *          from p restricted to the tokens not drawn yet).  Fewer than k tokens with p_v > 0
+ *          give -1 after them.
+ *   T == 0: the k largest logits, as eagle_draft_select.
+ * For the accept walk to keep the target distribution, each of these children must be given
+ * the row it was drawn from (eagle_draft_child_rows), not the parent's row.
+ */
+eagle_status_t eagle_draft_select_distinct(int32_t batch, int32_t rows_per_seq, int32_t vocab,
+                                           int32_t k, const float *logits, float temperature,
+                                           uint64_t seed, uint64_t offset, int32_t *tokens,
+                                           float *conf, float *probs, void *stream);
+
+/*
+ * The row each sibling drawn without replacement was drawn from (EAGLE summary, §2 and
+ * appendix A.2: the walk tests a child against the distribution that drafted it):
+ *   child_probs[b, f, j, v] = probs[b, f, v] / R_j  for v not in tokens[b, f, 0 .. j-1],
+ *                             0 otherwise,
+ *   R_j = the sum of probs[b, f, v] over those v (summed directly).  Row 0 is probs itself;
+ *   a token -1 (or >= V) before sibling j, or R_j = 0, makes row j all zeros.
+ *   probs [B, F, V] float32 device (eagle_draft_select_distinct's distribution output),
+ *   tokens [B, F, k] int32 device, child_probs [B, F, k, V] float32 device (written whole).
+ * 1 <= B <= 65535, 1 <= F <= 256, 1 <= k <= 16, V >= 1.  No workspace; one CTA per
+ * (row, sibling).
+ */
+eagle_status_t eagle_draft_child_rows(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
+                                      const float *probs, const int32_t *tokens,
+                                      float *child_probs, void *stream);
+
+/*
  * Reads (and, if `reset` != 0, clears) the device error word that bounded waits set
  * when they give up.  Synchronises the current device.  *code = 0 means no error.
  */

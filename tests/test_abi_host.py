@@ -169,6 +169,23 @@ def test_draft_select_checks_arguments_before_launch(lib):
     assert call(1, 4, 8 * 49152 + 1, 4) == binding.EAGLE_ERR_UNSUPPORTED
 
 
+def test_draft_distinct_and_child_rows_check_arguments_before_launch(lib):
+    call = lambda B, F, V, k, T=1.0, lg=FAKE: lib.eagle_draft_select_distinct(B, F, V, k, lg, T, 0, 0, FAKE,
+                                                                              FAKE, None, None)
+    assert call(1, 4, 1000, 17) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 8, 10) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 257, 1000, 4) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 1000, 4, T=float("inf")) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 1000, 4, lg=FAKE + 2) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert call(1, 4, 8 * 49152 + 1, 4) == binding.EAGLE_ERR_UNSUPPORTED
+    rows = lambda B, F, V, k, pr=FAKE, tk=FAKE, out=FAKE: lib.eagle_draft_child_rows(B, F, V, k, pr, tk, out, None)
+    assert rows(1, 4, 1000, 17) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert rows(0, 4, 1000, 4) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert rows(1, 4, 0, 4) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert rows(1, 4, 1000, 4, pr=None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+    assert rows(1, 4, 1000, 4, out=None) == binding.EAGLE_ERR_INVALID_ARGUMENT
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "nope.so"))
     monkeypatch.setattr(binding, "_lib", None)

@@ -24,6 +24,7 @@ DTYPE_BF16 = 1
 EXPORTED = ("eagle_status_string", "eagle_workspace_bytes", "eagle_tree_attention",
             "eagle_lm_head_logits", "eagle_tree_accept", "eagle_verify_step",
             "eagle_commit_accepted", "eagle_tree_rerank", "eagle_draft_select",
+            "eagle_draft_select_distinct", "eagle_draft_child_rows",
             "eagle_device_error")
 
 
@@ -82,6 +83,10 @@ def load() -> ctypes.CDLL:
     L.eagle_tree_rerank.argtypes = [i32, i32, i32] + [vp] * 9
     L.eagle_draft_select.restype = ctypes.c_int
     L.eagle_draft_select.argtypes = [i32, i32, i32, i32, vp, f32, u64, u64, vp, vp, vp, vp]
+    L.eagle_draft_select_distinct.restype = ctypes.c_int
+    L.eagle_draft_select_distinct.argtypes = [i32, i32, i32, i32, vp, f32, u64, u64, vp, vp, vp, vp]
+    L.eagle_draft_child_rows.restype = ctypes.c_int
+    L.eagle_draft_child_rows.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp]
     L.eagle_device_error.restype = ctypes.c_int
     L.eagle_device_error.argtypes = [ctypes.POINTER(i32), i32]
     _lib = L
@@ -184,6 +189,21 @@ def draft_select(logits, temperature: float, k: int, seed: int, offset: int, tok
     _check("eagle_draft_select", load().eagle_draft_select(
         int(B), int(F), int(V), int(k), _ptr(logits), float(temperature), int(seed), int(offset),
         _ptr(tokens), _ptr(conf), _ptr(probs), _stream(stream)))
+
+
+def draft_select_distinct(logits, temperature: float, k: int, seed: int, offset: int, tokens, conf,
+                          probs=None, stream=None) -> None:
+    B, F, V = logits.shape
+    _check("eagle_draft_select_distinct", load().eagle_draft_select_distinct(
+        int(B), int(F), int(V), int(k), _ptr(logits), float(temperature), int(seed), int(offset),
+        _ptr(tokens), _ptr(conf), _ptr(probs), _stream(stream)))
+
+
+def draft_child_rows(probs, tokens, child_probs, stream=None) -> None:
+    B, F, V = probs.shape
+    k = tokens.shape[-1]
+    _check("eagle_draft_child_rows", load().eagle_draft_child_rows(
+        int(B), int(F), int(V), int(k), _ptr(probs), _ptr(tokens), _ptr(child_probs), _stream(stream)))
 
 
 def device_error(reset: bool = True) -> int:

@@ -139,8 +139,32 @@ __device__ __forceinline__ void dsmem_st_s32(uint32_t addr, int v) {
   asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-template <bool kGreedy>
+// Kernel modes: the top k logits (T == 0), k independent races (T > 0, siblings drawn with
+// replacement), the k smallest keys of one race (T > 0, siblings drawn without replacement).
+constexpr int kDraftTopK = 0;
+constexpr int kDraftRaces = 1;
+constexpr int kDraftDistinct = 2;
+
+// Inserts (cv, ci) into a thread's list of its 16 best entries, sorted by draft_better.
+__device__ __forceinline__ void draft_list_insert(float (&lv)[kDraftMaxK], int (&li)[kDraftMaxK], float cv,
+                                                  int ci) {
+  if (!draft_better(cv, ci, lv[kDraftMaxK - 1], li[kDraftMaxK - 1])) return;
+#pragma unroll
+  for (int s = 0; s < kDraftMaxK; ++s)
+    if (draft_better(cv, ci, lv[s], li[s])) {  // carry the displaced entry down
+      const float tv = lv[s];
+      const int ti = li[s];
+      lv[s] = cv;
+      li[s] = ci;
+      cv = tv;
+      ci = ti;
+    }
+}
+
+template <int kMode>
 __global__ void __launch_bounds__(kDraftThreads) draft_select_kernel(const DraftParams p) {
+  constexpr bool kGreedy = kMode == kDraftTopK;
+  constexpr bool kList = kMode != kDraftRaces;  // winners from per-thread sorted lists
   __shared__ DraftShared sh;
   const uint32_t S = cluster_nctarank();
   const uint32_t cr = cluster_ctarank();
@@ -202,8 +226,10 @@ __global__ void __launch_bounds__(kDraftThreads) draft_select_kernel(const Draft
   const int lane = tid & 31, warp = tid >> 5;
   const uint32_t to0_v = dsmem_map(smem_u32(&sh.best_v[cr][0]), 0);
   const uint32_t to0_i = dsmem_map(smem_u32(&sh.best_i[cr][0]), 0);
-  if (kGreedy) {
-    // each thread's 16 best entries, sorted; NaN never enters (draft_better is false)
+  if (kList) {
+    // each thread's 16 best entries, sorted; NaN never enters (draft_better is false).  The
+    // value is the logit (top k) or the negated race key (without replacement: the k
+    // smallest keys of one race, purpose 2, are successive draws)
     float lv[kDraftMaxK];
     int li[kDraftMaxK];
 #pragma unroll
@@ -211,20 +237,19 @@ __global__ void __launch_bounds__(kDraftThreads) draft_select_kernel(const Draft
       lv[s] = -INFINITY;
       li[s] = INT_MAX;
     }
-    for (int i = tid; i < n; i += kDraftThreads) {
-      float cv = xs[i];
-      int ci = v_lo + i;
-      if (draft_better(cv, ci, lv[kDraftMaxK - 1], li[kDraftMaxK - 1])) {
+    if (kGreedy) {
+      for (int i = tid; i < n; i += kDraftThreads) draft_list_insert(lv, li, xs[i], v_lo + i);
+    } else {
+      for (int i0 = 4 * tid; i0 < n; i0 += 4 * kDraftThreads) {
+        const Philox4 u = philox_group(p.seed, p.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(f),
+                                       2u, static_cast<uint32_t>(v_lo + i0) >> 2);
 #pragma unroll
-        for (int s = 0; s < kDraftMaxK; ++s)
-          if (draft_better(cv, ci, lv[s], li[s])) {  // carry the displaced entry down
-            const float tv = lv[s];
-            const int ti = li[s];
-            lv[s] = cv;
-            li[s] = ci;
-            cv = tv;
-            ci = ti;
-          }
+        for (int e = 0; e < 4; ++e) {
+          if (i0 + e >= n) break;
+          const float lw = xs[i0 + e];
+          if (lw == -INFINITY) continue;
+          draft_list_insert(lv, li, lw - logf(-logf(word_to_uniform(u.w[e]))), v_lo + i0 + e);
+        }
       }
     }
     // the warp's k best: k rounds of a warp argmax over the lists' heads
@@ -331,7 +356,7 @@ __global__ void __launch_bounds__(kDraftThreads) draft_select_kernel(const Draft
 
   // CTA 0, warp 0: the row's k children; lane j writes child j
   int pick = INT_MAX;
-  if (kGreedy) {
+  if (kList) {
     int h = 0;  // lane s walks CTA s's list
     for (int j = 0; j < k; ++j) {
       const bool live = static_cast<uint32_t>(lane) < S && h < k;
@@ -354,6 +379,101 @@ __global__ void __launch_bounds__(kDraftThreads) draft_select_kernel(const Draft
     const bool found = pick != INT_MAX;
     p.tokens[static_cast<size_t>(r) * k + lane] = found ? pick : -1;
     p.conf[static_cast<size_t>(r) * k + lane] = found ? expf(row[pick] * invT - M) * invZ : 0.f;
+  }
+}
+
+// The row each sibling was drawn from, for siblings drawn without replacement: child j of
+// row r was drawn from p_r with tokens[r][0 .. j-1] removed, so its row is p_r over the rest,
+// renormalised by the remaining mass R_j summed directly over the kept entries (not 1 minus
+// the removed mass, which cancels when the earlier siblings carry most of it).
+//
+// A row is split over a cluster of C <= 8 CTAs, CTA c owning entries [c*W, (c+1)*W).  Each
+// entry v has a position pos(v) = i if v is sibling i's token, else k: it stays in rows
+// j <= pos(v).  Each CTA sums its entries into the k partial masses, pushes them into every
+// peer's shared memory, and after one hardware cluster barrier every CTA holds R_0..R_{k-1}
+// and writes its chunk of all k rows.  A token -1 (or out of range) before sibling j leaves
+// rows j.. all zeros.
+constexpr int kChildThreads = 512;
+constexpr int kChildMaxCluster = 8;
+
+struct ChildParams {
+  const float* probs;     // [R, V]
+  const int32_t* tokens;  // [R, k]
+  float* child;           // [R, k, V]
+  int32_t V, k, chunk;    // chunk: entries per CTA
+};
+
+__global__ void __launch_bounds__(kChildThreads) draft_child_rows_kernel(const ChildParams p) {
+  __shared__ int32_t tok[kDraftMaxK];
+  __shared__ float red[kChildThreads / 32][kDraftMaxK];
+  __shared__ float part[kChildMaxCluster][kDraftMaxK];  // CTA c's partial masses, pushed by c
+  const uint32_t C = cluster_nctarank();
+  const uint32_t cr = cluster_ctarank();
+  const int r = static_cast<int>(blockIdx.x / C);
+  const int V = p.V, k = p.k, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  if (tid < k) tok[tid] = p.tokens[static_cast<size_t>(r) * k + tid];
+  __syncthreads();
+  int live = k;  // rows j < live are defined: no -1 / out-of-range token before them
+  for (int i = 0; i < k; ++i)
+    if (tok[i] < 0 || tok[i] >= V) {
+      live = i + 1;  // row i itself is still defined (its earlier tokens are valid)
+      break;
+    }
+  const int v_lo = static_cast<int>(cr) * p.chunk;
+  const int v_hi = min(V, v_lo + p.chunk);
+  const float* row = p.probs + static_cast<size_t>(r) * V;
+  auto pos_of = [&](int v) {
+    int q = k;
+    for (int i = 0; i < k; ++i)
+      if (tok[i] == v) {
+        q = i;
+        break;
+      }
+    return q;
+  };
+
+  // this chunk's partial masses: entry v counts in rows j <= pos(v)
+  float acc[kDraftMaxK];
+#pragma unroll
+  for (int j = 0; j < kDraftMaxK; ++j) acc[j] = 0.f;
+  for (int v = v_lo + tid; v < v_hi; v += kChildThreads) {
+    const float x = row[v];
+    const int q = pos_of(v);
+#pragma unroll
+    for (int j = 0; j < kDraftMaxK; ++j)
+      if (j <= q) acc[j] += x;
+  }
+#pragma unroll
+  for (int j = 0; j < kDraftMaxK; ++j) {
+    float t = acc[j];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) red[warp][j] = t;
+  }
+  __syncthreads();
+  if (tid < k) {
+    float t = 0.f;
+    for (int w = 0; w < kChildThreads / 32; ++w) t += red[w][tid];
+    for (uint32_t c = 0; c < C; ++c) dsmem_st_f32(dsmem_map(smem_u32(&part[cr][tid]), c), t);
+  }
+  cluster_sync_all();  // the only exchange: no CTA reads a peer afterwards
+
+  float inv[kDraftMaxK];
+#pragma unroll
+  for (int j = 0; j < kDraftMaxK; ++j) {
+    float R = 0.f;
+    if (j < k)
+      for (uint32_t c = 0; c < C; ++c) R += part[c][j];
+    inv[j] = (j < live && R > 0.f) ? 1.0f / R : 0.f;
+  }
+  float* out = p.child + static_cast<size_t>(r) * k * V;
+  for (int v = v_lo + tid; v < v_hi; v += kChildThreads) {
+    const float x = row[v];
+    const int q = pos_of(v);
+#pragma unroll
+    for (int j = 0; j < kDraftMaxK; ++j)
+      if (j < k) out[static_cast<size_t>(j) * V + v] = (inv[j] == 0.f || q < j) ? 0.f : x * inv[j];
   }
 }
 

@@ -245,12 +245,12 @@ struct DeviceState {
   cudaEvent_t attn_done = nullptr;
   std::mutex step_mu;  // one step's fork/join sequence at a time on the shared side stream
   // eagle_draft_select: shared-memory limits set once; clusters of S CTAs resident at once,
-  // [greedy][log2 S][slice bytes in 4 KB steps], stored + 1 (0: not queried yet)
+  // [kernel mode][log2 S][slice bytes in 4 KB steps], stored + 1 (0: not queried yet)
   std::once_flag draft_once;
   bool draft_ok = false;
   int draft_max_cluster = kDraftPortableCluster;  // 16 where the device co-schedules them
   std::mutex draft_mu;
-  int draft_clusters[2][5][kDraftMaxSmem / 4096 + 1] = {};
+  int draft_clusters[3][5][kDraftMaxSmem / 4096 + 1] = {};
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -597,8 +597,15 @@ bool device_accept_supported(const eagle_shape_t* s, int dev) {
   return ap.nq >= 1 && ap.smem <= kAccMaxSmem;
 }
 
-template <bool kGreedy>
-int draft_active_clusters(int S, size_t smem) {
+const void* draft_kernel(int mode) {
+  switch (mode) {
+    case kDraftTopK: return reinterpret_cast<const void*>(draft_select_kernel<kDraftTopK>);
+    case kDraftRaces: return reinterpret_cast<const void*>(draft_select_kernel<kDraftRaces>);
+    default: return reinterpret_cast<const void*>(draft_select_kernel<kDraftDistinct>);
+  }
+}
+
+int draft_active_clusters(int mode, int S, size_t smem) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(S));
   cfg.blockDim = dim3(kDraftThreads);
@@ -611,7 +618,7 @@ int draft_active_clusters(int S, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, draft_select_kernel<kGreedy>, &cfg) != cudaSuccess) n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, draft_kernel(mode), &cfg) != cudaSuccess) n = 0;
   cudaGetLastError();
   return n;
 }
@@ -623,7 +630,7 @@ int draft_slice(int V, int S) { return (((V + S - 1) / S + 3) / 4) * 4; }
 // the largest S in {16, 8, 4, 2} whose clusters are all resident at once, with slices of at
 // least 1024 entries; else the smallest S whose slice fits (more rows than one wave holds
 // gain nothing from splitting).  0: no S fits.
-int draft_cluster(int dev, long rows, int V, bool greedy) {
+int draft_cluster(int dev, long rows, int V, int mode) {
   DeviceState& ds = g_dev[dev];
   int first_fit = 0;
   for (int lg = 0; lg < 4; ++lg) {  // portable sizes only
@@ -642,10 +649,8 @@ int draft_cluster(int dev, long rows, int V, bool greedy) {
     int n;
     {
       std::lock_guard<std::mutex> lock(ds.draft_mu);
-      int& slot = ds.draft_clusters[greedy ? 1 : 0][lg][bucket];
-      if (slot == 0)
-        slot = 1 + (greedy ? draft_active_clusters<true>(S, bucket * 4096)
-                           : draft_active_clusters<false>(S, bucket * 4096));
+      int& slot = ds.draft_clusters[mode][lg][bucket];
+      if (slot == 0) slot = 1 + draft_active_clusters(mode, S, bucket * 4096);
       n = slot - 1;
     }
     if (rows <= n) return S;
@@ -657,19 +662,62 @@ bool ensure_draft(int dev) {
   DeviceState& ds = g_dev[dev];
   std::call_once(ds.draft_once, [&] {
     const int bytes = static_cast<int>(kDraftMaxSmem);
-    ds.draft_ok = cudaFuncSetAttribute(draft_select_kernel<true>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
-                  cudaFuncSetAttribute(draft_select_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
-    if (cudaFuncSetAttribute(draft_select_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-            cudaSuccess &&
-        cudaFuncSetAttribute(draft_select_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-            cudaSuccess &&
-        draft_active_clusters<true>(16, 4096) >= 1 && draft_active_clusters<false>(16, 4096) >= 1)
-      ds.draft_max_cluster = 16;
+    bool ok = true, wide = true;
+    for (int mode = 0; mode < 3; ++mode) {
+      ok &= cudaFuncSetAttribute(draft_kernel(mode), cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+            cudaSuccess;
+      wide &= cudaFuncSetAttribute(draft_kernel(mode), cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+              cudaSuccess;
+    }
+    for (int mode = 0; mode < 3 && wide; ++mode) wide &= draft_active_clusters(mode, 16, 4096) >= 1;
+    ds.draft_ok = ok;
+    if (wide) ds.draft_max_cluster = 16;
     cudaGetLastError();
   });
   return ds.draft_ok;
+}
+
+// eagle_draft_select / eagle_draft_select_distinct: argument checks, then one cluster launch.
+eagle_status_t draft_launch(int mode, int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
+                            const float* logits, float temperature, uint64_t seed, uint64_t offset,
+                            int32_t* tokens, float* conf, float* probs, void* stream) {
+  if (batch < 1 || batch > 65535 || rows_per_seq < 1 || rows_per_seq > 256 || k < 1 ||
+      k > kDraftMaxK || vocab < k)
+    return EAGLE_ERR_INVALID_ARGUMENT;
+  if (!(temperature >= 0.f) || !std::isfinite(temperature)) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (logits == nullptr || tokens == nullptr || conf == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(logits) & 3) != 0) return EAGLE_ERR_INVALID_ARGUMENT;
+  if (static_cast<size_t>(draft_slice(vocab, kDraftPortableCluster)) * 4 > kDraftMaxSmem)
+    return EAGLE_ERR_UNSUPPORTED;  // a row must fit the shared memory of one cluster
+  if (temperature == 0.f) mode = kDraftTopK;
+  int dev;
+  if (!current_device(&dev) || !ensure_draft(dev)) return EAGLE_ERR_CUDA;
+  const long rows = static_cast<long>(batch) * rows_per_seq;
+  const int S = draft_cluster(dev, rows, vocab, mode);
+  if (S == 0) return EAGLE_ERR_UNSUPPORTED;
+  const int slice = draft_slice(vocab, S);
+  const int vec16 = (vocab % 4 == 0 && aligned16(logits)) ? 1 : 0;
+  DraftParams p{logits, tokens, conf, probs, rows_per_seq, vocab, k, slice, vec16, temperature, seed, offset};
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * S));
+  cfg.blockDim = dim3(kDraftThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(slice) * 4;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  switch (mode) {
+    case kDraftTopK: e = cudaLaunchKernelEx(&cfg, draft_select_kernel<kDraftTopK>, p); break;
+    case kDraftRaces: e = cudaLaunchKernelEx(&cfg, draft_select_kernel<kDraftRaces>, p); break;
+    default: e = cudaLaunchKernelEx(&cfg, draft_select_kernel<kDraftDistinct>, p); break;
+  }
+  if (e != cudaSuccess) return EAGLE_ERR_CUDA;
+  return launch_status();
 }
 
 }  // namespace
@@ -830,38 +878,42 @@ eagle_status_t eagle_draft_select(int32_t batch, int32_t rows_per_seq, int32_t v
                                   const float* logits, float temperature, uint64_t seed,
                                   uint64_t offset, int32_t* tokens, float* conf, float* probs,
                                   void* stream) {
+  return draft_launch(kDraftRaces, batch, rows_per_seq, vocab, k, logits, temperature, seed, offset,
+                      tokens, conf, probs, stream);
+}
+
+eagle_status_t eagle_draft_select_distinct(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
+                                           const float* logits, float temperature, uint64_t seed,
+                                           uint64_t offset, int32_t* tokens, float* conf, float* probs,
+                                           void* stream) {
+  return draft_launch(kDraftDistinct, batch, rows_per_seq, vocab, k, logits, temperature, seed, offset,
+                      tokens, conf, probs, stream);
+}
+
+eagle_status_t eagle_draft_child_rows(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
+                                      const float* probs, const int32_t* tokens, float* child_probs,
+                                      void* stream) {
   if (batch < 1 || batch > 65535 || rows_per_seq < 1 || rows_per_seq > 256 || k < 1 ||
-      k > kDraftMaxK || vocab < k)
+      k > kDraftMaxK || vocab < 1)
     return EAGLE_ERR_INVALID_ARGUMENT;
-  if (!(temperature >= 0.f) || !std::isfinite(temperature)) return EAGLE_ERR_INVALID_ARGUMENT;
-  if (logits == nullptr || tokens == nullptr || conf == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
-  if ((reinterpret_cast<uintptr_t>(logits) & 3) != 0) return EAGLE_ERR_INVALID_ARGUMENT;
-  if (static_cast<size_t>(draft_slice(vocab, kDraftPortableCluster)) * 4 > kDraftMaxSmem)
-    return EAGLE_ERR_UNSUPPORTED;  // a row must fit the shared memory of one cluster
-  int dev;
-  if (!current_device(&dev) || !ensure_draft(dev)) return EAGLE_ERR_CUDA;
+  if (probs == nullptr || tokens == nullptr || child_probs == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
   const long rows = static_cast<long>(batch) * rows_per_seq;
-  const bool greedy = temperature == 0.f;
-  const int S = draft_cluster(dev, rows, vocab, greedy);
-  if (S == 0) return EAGLE_ERR_UNSUPPORTED;
-  const int slice = draft_slice(vocab, S);
-  const int vec16 = (vocab % 4 == 0 && aligned16(logits)) ? 1 : 0;
-  DraftParams p{logits, tokens, conf, probs, rows_per_seq, vocab, k, slice, vec16, temperature, seed, offset};
+  int C = (vocab + 4095) / 4096;  // chunks of at least 4096 entries, up to 8 per row
+  if (C > kChildMaxCluster) C = kChildMaxCluster;
+  if (C < 1) C = 1;
+  ChildParams p{probs, tokens, child_probs, vocab, k, (vocab + C - 1) / C};
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(rows * S));
-  cfg.blockDim = dim3(kDraftThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(slice) * 4;
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * C));
+  cfg.blockDim = dim3(kChildThreads);
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = greedy ? cudaLaunchKernelEx(&cfg, draft_select_kernel<true>, p)
-                               : cudaLaunchKernelEx(&cfg, draft_select_kernel<false>, p);
-  if (e != cudaSuccess) return EAGLE_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, draft_child_rows_kernel, p) != cudaSuccess) return EAGLE_ERR_CUDA;
   return launch_status();
 }
 

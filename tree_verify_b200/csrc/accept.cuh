@@ -510,9 +510,9 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     prm.accept_len[b] = nacc;
     prm.next_token[b] = next;
   }
-  // Every peer's pushes into this CTA were awaited in the last reduction, and every remote
-  // read of a residual entry precedes its reader's next push, so no peer can still touch
-  // this CTA's shared memory: no closing cluster barrier is needed.
+  // Every CTA takes the same reductions, and a CTA's last one waited for every peer's push
+  // into its shared memory (peers only push, they never load from it), so no peer can still
+  // touch this CTA's shared memory: no closing cluster barrier is needed.
 }
 
 }  // namespace eagle

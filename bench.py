@@ -273,7 +273,9 @@ def main():
 
     # ---- the same step replayed from a CUDA graph (one fixed seed/offset per capture),
     # timed the same way: what launch gaps cost the stream-launched step
-    graph_info = {}
+    # Capture may fail on a rank (it is reported, never required); every rank still takes
+    # the same barriers, timing the stream-launched step in its place.
+    graph, graph_err = None, None
     try:
         gstream = torch.cuda.Stream(dev)
         gstream.wait_stream(stream)
@@ -284,23 +286,27 @@ def main():
             with torch.cuda.graph(graph, stream=gstream):
                 step.run(x, T, seed=rank, offset=0, stream=gstream)
         stream.wait_stream(gstream)
-        gs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ge = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        barrier()
-        for i in range(args.steps):
-            l2_flush()
-            gs[i].record(stream)
+    except Exception as exc:
+        graph, graph_err = None, f"{type(exc).__name__}: {exc}"[:200]
+    torch.cuda.synchronize(dev)
+    gs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ge = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        l2_flush()
+        gs[i].record(stream)
+        if graph is not None:
             graph.replay()
-            ge[i].record(stream)
-        barrier()
-        graph_ms = float(np.mean([s_.elapsed_time(e_) for s_, e_ in zip(gs, ge)]))
-        assert binding.device_error(reset=True) == 0
-        graph_info = {"ms_per_step": graph_ms, "value": world / (graph_ms / 1e3),
-                      "note": "eagle_verify_step captured once (seed rank, offset 0) and replayed"}
-        del graph
-    except Exception as exc:  # capture is reported, never required
-        graph_info = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
-        torch.cuda.synchronize(dev)
+        else:
+            step.run(x, T, seed=rank, offset=0)
+        ge[i].record(stream)
+    barrier()
+    graph_ms = float(np.mean([s_.elapsed_time(e_) for s_, e_ in zip(gs, ge)]))
+    assert binding.device_error(reset=True) == 0
+    graph_info = ({"ms_per_step": graph_ms, "value": world / (graph_ms / 1e3),
+                   "note": "eagle_verify_step captured once (seed rank, offset 0) and replayed"}
+                  if graph_err is None else {"unavailable": graph_err})
+    del graph
 
     # ---- dominant kernel alone (LM head), same conditions, for the roofline
     ls = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -445,10 +451,12 @@ def main():
         barrier()
         return float(np.mean([s.elapsed_time(e) for s, e in zip(ss_, se_)]))
     stacked_launch_ms = timed(stacked_pass)
-    stacked_ms = timed(stacked_graph.replay) if stacked_graph is not None else stacked_launch_ms
+    # the same number of barriers on every rank, graph or not
+    stacked_ms = timed(stacked_graph.replay if stacked_graph is not None else stacked_pass)
     assert binding.device_error(reset=True) == 0
     lens_h = x.prefix_lens.cpu().numpy().astype(np.int64)
     stacked_kv = int(STACK_LAYERS * lens_h.sum() * w.num_kv_heads * w.head_dim * 2 * x.k_prefix.element_size())
+    stacked_graph_ok = stacked_graph is not None
     del stacked_graph
     del st_q, st_kp, st_vp, st_kt, st_vt, st_out
 
@@ -527,8 +535,8 @@ def main():
                                        "own caches per layer",
                            "layers": STACK_LAYERS, "us_per_pass": stacked_ms * 1e3,
                            "us_per_pass_launched": stacked_launch_ms * 1e3,
-                           "timing": "CUDA graph replay of the pass" if stacked_ms != stacked_launch_ms
-                                     else "stream-launched",
+                           "timing": "CUDA graph replay of the pass" if stacked_graph_ok
+                                     else "stream-launched (capture failed)",
                            "us_per_layer": stacked_ms * 1e3 / STACK_LAYERS,
                            "prefix_kv_bytes_per_pass": stacked_kv,
                            "achieved_gbs": stacked_kv / (stacked_ms / 1e3) / 1e9,

@@ -39,6 +39,15 @@
  *                        a node is reached only if its whole path is accepted, so its
  *                        value is the product of the confidences along the path; the
  *                        m highest-valued candidates form the verified tree.
+ *   O6 draft children   (EAGLE summary, appendix A.1 "Tree Structure": in greedy decoding
+ *                        a node's children are the top k tokens, otherwise k tokens are
+ *                        sampled): the top k logits at T == 0, k independent races over
+ *                        softmax(logits / T) at T > 0, each child's probability as its
+ *                        confidence.
+ *   O7 without replacement (the same passage, siblings kept distinct): the k smallest
+ *                        clocks of one race, in order (successive draws), and the row
+ *                        each sibling was drawn from (the parent's row without the
+ *                        earlier siblings, renormalised).
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - the adjusted distribution is norm(max(0, p - p_hat)) (standard speculative
@@ -58,12 +67,17 @@
  *     numbers: as easy as 1, 2, 3", SC'11) with key = seed and counter
  *     (v >> 2, b << 16 | purpose << 8 | node, offset_lo, offset_hi); word v & 3;
  *     U = (2 * (x >> 9) + 1) * 2^-24.  The accept test of candidate c uses
- *     (node c, v 0, purpose 0); the race at node n uses (node n, v, purpose 1).
+ *     (node c, v 0, purpose 0); the race at node n uses (node n, v, purpose 1); draft
+ *     node f's race j (O6) uses (node f, v, purpose 2 + j), and O7's one race purpose 2.
  *
  * Parity pins live in the not-gpu tests: brute-force path attention and torch's
  * causal SDPA in float64 (O1), numpy float64 matmul (O2), brute-force argmax path
  * matching at T = 0 and chi-square tests of the emitted-token distribution, the
- * closed-form single-candidate acceptance probability and the race sampler (O3).
+ * closed-form single-candidate acceptance probability and the race sampler (O3);
+ * SDPA over the committed cache (O4); closed forms, value dominance and transitive
+ * closure (O5); numpy argsort and scipy softmax, chi-square and independence (O6); the
+ * law of successive draws, numpy renormalisation and the chi-square study of the
+ * residual rule with and without each sibling's own row (O7).
  */
 #include <math.h>
 #include <stdint.h>

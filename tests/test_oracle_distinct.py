@@ -123,3 +123,19 @@ def test_residual_rule_with_shared_rows_does_not(orc, q_logits, p_logits, k):
     counts = _first_emitted(orc, q_logits, p_logits, k, conditioned=False)
     p = _p(p_logits)
     assert stats.chisquare(counts, counts.sum() * p).pvalue < 1e-6
+
+
+def test_child_rows_sum_the_remaining_mass_directly(orc):
+    """When the earlier siblings carry all but ~1e-9 of the mass, 1 minus their mass loses
+    most of the digits of what remains; the rows must still be the exact renormalisation."""
+    V, k = 64, 3
+    p = np.full(V, 1e-11)
+    p[[5, 9]] = 0.5 - 16e-11
+    p /= p.sum()
+    tokens = np.array([[[5, 9, 2]]], np.int32)
+    rows = orc.draft_child_rows(p[None, None], tokens)
+    rest = np.delete(np.arange(V), [5, 9])
+    want = np.zeros(V)
+    want[rest] = p[rest] / p[rest].sum()
+    np.testing.assert_allclose(rows[0, 0, 2], want, rtol=1e-12, atol=0)
+    assert abs(rows[0, 0, 2].sum() - 1.0) < 1e-12

@@ -83,7 +83,7 @@ def lib() -> ctypes.CDLL:
                                ctypes.c_int32, ctypes.c_int32, vp]
         L.orc_tree_accept.argtypes = ([ctypes.c_int] * 4 + [vp, ctypes.c_int, ctypes.c_int,
                                       vp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_uint64,
-                                      ctypes.c_uint64, ctypes.c_double] + [vp] * 6)
+                                      ctypes.c_uint64, ctypes.c_double] + [vp] * 8)
         L.orc_num_threads.restype = ctypes.c_int
         L.orc_fill_uniforms.argtypes = [ctypes.c_uint64, ctypes.c_uint64] + [ctypes.c_int32] * 4 + [vp]
         del i32p, f64p
@@ -185,7 +185,11 @@ def tree_accept(draft_probs, tokens, parents, temperature: float, seed: int = 0,
                 offset: int = 0, logits=None, hidden=None, w_lm=None, margin: float = 1e-4):
     """O3.  ``logits`` [B,N,V] (float32 or float64), or ``hidden``/``w_lm`` to let the
     oracle compute the rows it visits.  Returns a dict with accepted_nodes [B,N],
-    accept_len [B], next_token [B] and the margin diagnostics near/decisions/first_near."""
+    accept_len [B], next_token [B] and the margin diagnostics [B]: near (decisions inside
+    the margin), decisions, first_near (index of the first near decision, -1 if none),
+    exact_len (accepted nodes fixed before it; accept_len when there is none) and
+    near_child (the candidate tested at the first near decision; -1 when it is the final
+    race or there is none, -2 when it is a greedy argmax)."""
     B, N, V = draft_probs.shape
     dp = np.ascontiguousarray(draft_probs, dtype=np.float32)
     tk = np.ascontiguousarray(tokens, dtype=np.int32)
@@ -209,13 +213,16 @@ def tree_accept(draft_probs, tokens, parents, temperature: float, seed: int = 0,
     near = np.zeros(B, dtype=np.int32)
     ndec = np.zeros(B, dtype=np.int32)
     first = np.zeros(B, dtype=np.int32)
+    exact_len = np.zeros(B, dtype=np.int32)
+    near_child = np.zeros(B, dtype=np.int32)
     rc = lib().orc_tree_accept(B, N, V, mode, lp, H, et, hp, wp, _p(dp), _p(tk), _p(par),
                                float(temperature), seed, offset, float(margin), _p(acc),
-                               _p(alen), _p(nxt), _p(near), _p(ndec), _p(first))
+                               _p(alen), _p(nxt), _p(near), _p(ndec), _p(first),
+                               _p(exact_len), _p(near_child))
     if rc != OK:
         raise ValueError(f"oracle tree_accept rejected its inputs (code {rc})")
     return dict(accepted_nodes=acc, accept_len=alen, next_token=nxt, near=near,
-                decisions=ndec, first_near=first)
+                decisions=ndec, first_near=first, exact_len=exact_len, near_child=near_child)
 
 
 def commit(k_prefix, v_prefix, prefix_lens, k_tree, v_tree, hidden, parents, accepted_nodes,

@@ -352,15 +352,25 @@ static void orc_get_row(const orc_rows_t *src, int b, int node, double *row)
 }
 
 typedef struct {
-    int32_t near;     /* decisions within the margin */
+    int32_t near;       /* decisions within the margin */
     int32_t decisions;
     int32_t first_near; /* index of the first near decision, -1 if none */
+    int32_t exact_len;  /* accepted nodes fixed before the first near decision */
+    int32_t near_child; /* the child tested at the first near decision; -1 when that decision
+                           is the final race or when there is none, -2 when it is a greedy
+                           argmax (which decides both the match and the final token) */
 } orc_diag_t;
 
-static void orc_note(orc_diag_t *dg, int is_near)
+/* Records one decision of the walk: `n_acc` nodes accepted so far, `child` the candidate
+ * under test (-1 for the argmax or race that ends the walk). */
+static void orc_note(orc_diag_t *dg, int is_near, int n_acc, int child)
 {
     if (is_near) {
-        if (dg->near == 0) dg->first_near = dg->decisions;
+        if (dg->near == 0) {
+            dg->first_near = dg->decisions;
+            dg->exact_len = n_acc;
+            dg->near_child = child;
+        }
         dg->near++;
     }
     dg->decisions++;
@@ -389,7 +399,7 @@ static int orc_walk(const orc_rows_t *src, int b, int N, int V, const float *dra
             double second = -INFINITY;
             for (int v = 0; v < V; ++v)
                 if (v != m && logit_row[v] > second) second = logit_row[v];
-            orc_note(dg, V > 1 && logit_row[m] - second <= margin);
+            orc_note(dg, V > 1 && logit_row[m] - second <= margin, n_acc, -2);
             int matched = -1;
             for (int c = cur + 1; c < N; ++c)
                 if (parents_b[c] == cur && tokens_b[c] == m) {
@@ -423,12 +433,12 @@ static int orc_walk(const orc_rows_t *src, int b, int N, int V, const float *dra
             const float *p_hat = draft_b + (size_t)c * V;
             const double u = orc_uniform(seed, offset, b, c, 0, 0);
             if (p_hat[t_hat] == 0.0f) {
-                orc_note(dg, 0);
+                orc_note(dg, 0, n_acc, c);
                 accepted = c;
                 break;
             }
             const double ratio = p[t_hat] / (double)p_hat[t_hat];
-            orc_note(dg, fabs(u - ratio) <= margin * (ratio > 1.0 ? ratio : 1.0));
+            orc_note(dg, fabs(u - ratio) <= margin * (ratio > 1.0 ? ratio : 1.0), n_acc, c);
             if (u < ratio) {
                 accepted = c;
                 break;
@@ -450,7 +460,7 @@ static int orc_walk(const orc_rows_t *src, int b, int N, int V, const float *dra
         }
         double gap;
         *next_token = orc_race(V, p, seed, offset, b, cur, &gap);
-        orc_note(dg, gap <= margin);
+        orc_note(dg, gap <= margin, n_acc, -1);
         return n_acc;
     }
 }
@@ -458,13 +468,16 @@ static int orc_walk(const orc_rows_t *src, int b, int N, int V, const float *dra
 /* logits_mode 0: `logits` is float [B,N,V]; 1: double [B,N,V]; 2: rows are computed on
  * demand from hidden [B*N,H] and w [V,H] (elem_type).  Outputs: accepted_nodes [B,N]
  * (-1 padded), accept_len [B] and next_token [B] (-1 and -1 for an invalid tree);
- * diagnostics (may be NULL): near_count, n_decisions, first_near per sequence. */
+ * diagnostics (may be NULL), per sequence: near_count, n_decisions, first_near, and for
+ * the first near decision exact_len (accepted nodes fixed before it) and near_child (the
+ * candidate it tested; -1 for the final race or none, -2 for a greedy argmax). */
 int orc_tree_accept(int B, int N, int V, int logits_mode, const void *logits, int H,
                     int elem_type, const void *hidden, const void *w, const float *draft_probs,
                     const int32_t *tokens, const int32_t *parents, double temperature,
                     uint64_t seed, uint64_t offset, double margin, int32_t *accepted_nodes,
                     int32_t *accept_len, int32_t *next_token, int32_t *near_count,
-                    int32_t *n_decisions, int32_t *first_near)
+                    int32_t *n_decisions, int32_t *first_near, int32_t *exact_len,
+                    int32_t *near_child)
 {
     if (B < 1 || B > 65535 || N < 1 || N > 64 || V < 1 || !(temperature >= 0.0))
         return ORC_BAD_ARG;
@@ -478,7 +491,7 @@ int orc_tree_accept(int B, int N, int V, int logits_mode, const void *logits, in
         for (int b = 0; b < B; ++b) {
             int32_t *acc = accepted_nodes + (size_t)b * N;
             for (int i = 0; i < N; ++i) acc[i] = -1;
-            orc_diag_t dg = {0, 0, -1};
+            orc_diag_t dg = {0, 0, -1, 0, -1};
             int32_t nt = -1;
             const int n = orc_walk(&src, b, N, V, draft_probs + (size_t)b * N * V,
                                    tokens + (size_t)b * N, parents + (size_t)b * N,
@@ -488,6 +501,8 @@ int orc_tree_accept(int B, int N, int V, int logits_mode, const void *logits, in
             if (near_count) near_count[b] = dg.near;
             if (n_decisions) n_decisions[b] = dg.decisions;
             if (first_near) first_near[b] = dg.first_near;
+            if (exact_len) exact_len[b] = dg.near > 0 ? dg.exact_len : (n < 0 ? 0 : n);
+            if (near_child) near_child[b] = dg.near_child;
         }
         free(row);
         free(p);

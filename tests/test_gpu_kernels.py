@@ -198,8 +198,11 @@ def test_tree_accept_matches_oracle(cuda_lib, orc, T, V):
         got = _run_accept(cuda_lib, logits, draft, tokens, par, T, seed, offset)
         ref = orc.tree_accept(draft, tokens, par, T, seed=seed, offset=offset, logits=logits,
                               margin=MARGIN)
-        exact = compare_accept(got, ref, par, exact_all=(T == 0.0))
-        assert exact >= B - 2
+        st = compare_accept(got, ref, par, exact_all=(T == 0.0))
+        # identical fp32 logits on both sides: at T = 0 every decision is compared; at T > 0
+        # only decisions inside the margin (rare at these sizes) are excluded
+        assert st.compared >= 0.95 * st.decisions, st
+        assert st.whole >= B - 2, st
     # the walks are not trivial
     assert ref["accept_len"].max() >= 2
 
@@ -210,7 +213,8 @@ def test_tree_accept_large_vocab(cuda_lib, orc):
     logits, draft, tokens, par = _accept_inputs(rng, B, N, V, 1.0)
     got = _run_accept(cuda_lib, logits, draft, tokens, par, 1.0, 5, 6)
     ref = orc.tree_accept(draft, tokens, par, 1.0, seed=5, offset=6, logits=logits)
-    assert compare_accept(got, ref, par) >= B - 1
+    st = compare_accept(got, ref, par)
+    assert st.compared >= 0.9 * st.decisions, st
 
 
 def test_tree_accept_invalid_trees(cuda_lib):

@@ -52,9 +52,11 @@ _lib: Optional[ctypes.CDLL] = None
 
 
 def lib() -> ctypes.CDLL:
+    """The compiled oracle.  EAGLE_ORACLE_LIB names another build of oracle.c to load
+    instead (the mutation tests load deliberately broken copies this way)."""
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        _lib = ctypes.CDLL(os.environ.get("EAGLE_ORACLE_LIB") or build())
         L = _lib
         vp, i32p, f64p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p
         L.orc_uniform.restype = ctypes.c_double

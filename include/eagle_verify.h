@@ -24,6 +24,15 @@
  *   - Device-side waits are bounded.  If one gives up (a hardware stall, never a
  *     normal run) the kernel records a code readable with eagle_device_error().
  *   - No C++ exception crosses this boundary.
+ *   - State the library keeps (a departure from "no global state"): per device, the
+ *     kernels' shared-memory and cluster attributes (set once), eagle_verify_step's second
+ *     stream with two events and a host mutex (created on the first bf16 call; bf16 steps
+ *     on one device are enqueued one at a time), the occupancy answers the draft kernels
+ *     plan with, the fixed scratch array of eagle_tree_attention_static, and ONE device
+ *     error word shared by every call and stream (first writer wins; eagle_device_error
+ *     synchronises the device to read it).  Calls on different streams with different
+ *     workspaces compute independently; only the error word and the step's side stream
+ *     are shared.
  *
  * Shape symbols: B batch, N tree rows per sequence (root node 0 included, <= 64),
  * Hq / Hkv query / key-value heads (G = Hq / Hkv), D head_dim (64 or 128),
@@ -84,7 +93,8 @@ size_t eagle_workspace_bytes(const eagle_shape_t *shape);
  *   q            [B,N,Hq,D]       dtype
  *   k_prefix     [B,Hkv,Lmax,D]   dtype; positions >= prefix_lens[b] are never read
  *   v_prefix     [B,Hkv,Lmax,D]   dtype
- *   prefix_lens  [B] int32, each in 0..Lmax
+ *   prefix_lens  [B] int32, each in 0..Lmax (a value outside is clamped into that range
+ *                and recorded as device error 0x205)
  *   k_tree       [B,N,Hkv,D]      dtype; keys of the tree nodes (post-RoPE)
  *   v_tree       [B,N,Hkv,D]      dtype
  *   parents      [B,N] int32: parents[b,0] = -1, 0 <= parents[b,i] < i
@@ -136,6 +146,12 @@ eagle_status_t eagle_lm_head_logits(const eagle_shape_t *shape, const void *hidd
  *   accepted_nodes  [B,N] int32 out: accepted drafted nodes root-to-leaf, -1 padded
  *   accept_len      [B] int32 out: number of accepted nodes, -1 for an invalid tree
  *   next_token      [B] int32 out: the one extra emitted token, -1 for an invalid tree
+ * One thread-block cluster walks a sequence, its CTAs splitting the vocabulary and
+ * exchanging partials through distributed shared memory; every exchange carries what it is
+ * about, and if the CTAs of a cluster ever disagreed (or a bounded wait gave up) they stop
+ * together: that sequence then reports accept_len = next_token = -1 like an invalid tree
+ * and the device error word says why (0x303: the CTAs disagreed; 0x301 / 0x302: a wait
+ * gave up).  Node indices (< 64) and the purposes (0, 1) fit the counter's 8-bit fields.
  *   workspace       as for eagle_tree_attention (unused today; pass the same buffer)
  */
 eagle_status_t eagle_tree_accept(const eagle_shape_t *shape, const float *logits,
@@ -191,7 +207,9 @@ eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
  * two calls whose work overlaps on the GPU (different streams, or different host threads)
  * race on it and must be ordered by the caller.  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture.  This entry point allocates nothing.
+ * first call before any stream capture.  A lookup that fails returns EAGLE_ERR_CUDA and is
+ * not remembered: the next call on that device tries again.  This entry point allocates
+ * nothing.
  */
 #define EAGLE_STATIC_SCRATCH_BYTES (16u << 20)
 eagle_status_t eagle_tree_attention_static(const eagle_shape_t *shape, const void *q,
@@ -281,9 +299,11 @@ eagle_status_t eagle_tree_rerank(int32_t batch, int32_t num_candidates, int32_t 
  *   logits  [B, F, V] float32 device;  tokens [B, F, k] int32;  conf [B, F, k] float32;
  *   probs   [B, F, V] float32 or NULL
  * 1 <= B <= 65535, 1 <= F (rows_per_seq) <= 256, 1 <= k <= 16, k <= V, T >= 0 finite,
- * logits 4-byte aligned (else EAGLE_ERR_INVALID_ARGUMENT).  A row is split over a cluster of
- * up to 8 CTAs, each holding its slice in shared memory, so V <= 393216 (else
- * EAGLE_ERR_UNSUPPORTED).  No workspace.
+ * logits 4-byte aligned (else EAGLE_ERR_INVALID_ARGUMENT).  The row index f and the purpose
+ * 2 + j each fill 8 bits of the Philox counter, which these bounds keep them within.  A row
+ * is split over a thread-block cluster of up to 16 CTAs (16 where the device co-schedules
+ * them, else up to 8), each holding its slice in shared memory; a row must fit 8 slices of
+ * 192 KB, so V <= 393216 (else EAGLE_ERR_UNSUPPORTED).  No workspace.
  */
 eagle_status_t eagle_draft_select(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
                                   const float *logits, float temperature, uint64_t seed,
@@ -317,8 +337,9 @@ eagle_status_t eagle_draft_select_distinct(int32_t batch, int32_t rows_per_seq, 
  *   a token -1 (or >= V) before sibling j, or R_j = 0, makes row j all zeros.
  *   probs [B, F, V] float32 device (eagle_draft_select_distinct's distribution output),
  *   tokens [B, F, k] int32 device, child_probs [B, F, k, V] float32 device (written whole).
- * 1 <= B <= 65535, 1 <= F <= 256, 1 <= k <= 16, V >= 1.  No workspace; one CTA per
- * (row, sibling).
+ * 1 <= B <= 65535, 1 <= F <= 256, 1 <= k <= 16, V >= 1.  No workspace.  A row is split
+ * over a thread-block cluster of up to 8 CTAs (chunks of at least 4096 entries), each of
+ * which writes its chunk of all k rows.
  */
 eagle_status_t eagle_draft_child_rows(int32_t batch, int32_t rows_per_seq, int32_t vocab, int32_t k,
                                       const float *probs, const int32_t *tokens,
@@ -327,6 +348,10 @@ eagle_status_t eagle_draft_child_rows(int32_t batch, int32_t rows_per_seq, int32
 /*
  * Reads (and, if `reset` != 0, clears) the device error word that bounded waits set
  * when they give up.  Synchronises the current device.  *code = 0 means no error.
+ * Codes: 0x101-0x103 an LM-head wait gave up; 0x201-0x203 a tree-attention wait gave up;
+ * 0x204 a launch plan gave a compact attention CTA two tiles; 0x205 a prefix length
+ * outside [0, Lmax] (clamped); 0x301 / 0x302 an accept-walk copy / cluster wait gave up;
+ * 0x303 the CTAs of an accept-walk cluster disagreed and stopped.
  */
 eagle_status_t eagle_device_error(int32_t *code, int32_t reset);
 

@@ -105,6 +105,22 @@ def test_tree_attention_invalid_parent_is_safe(cuda_lib, orc):
     assert row_rel_err(got[0, ok_rows], ref[0, ok_rows]).max() <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_tree_attention_out_of_range_prefix_len_is_recorded(cuda_lib, orc, dtype):
+    """A prefix length outside [0, Lmax] is a caller bug the host cannot see (the lengths
+    live on the device): the kernel clamps it into range, so it stays in bounds, and
+    records device error 0x205."""
+    rng = np.random.default_rng(21)
+    inp = _attn_case(rng, 2, 5, 4, 2, 128, 100, [100, 40], dtype)
+    inp["prefix_lens"] = np.asarray([250, -3], np.int32)
+    got = _run_attention(cuda_lib, inp, dtype)
+    assert cuda_lib.device_error(reset=True) == 0x205
+    ref = orc.tree_attention(**dict(inp, prefix_lens=np.asarray([100, 0], np.int32)))
+    assert np.isfinite(got[0]).all()
+    assert row_rel_err(got[0], ref[0]).max() <= TOL[dtype]
+    assert row_rel_err(got[1], ref[1]).max() <= TOL[dtype]
+
+
 def _path(par, i):
     out = []
     while i >= 0:

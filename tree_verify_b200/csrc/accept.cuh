@@ -94,10 +94,22 @@ struct OpSum {  // (sum, owner fields)
   }
 };
 
+// What a reduction is about, pushed beside its partial: (site << 24) | (node << 16) |
+// (candidate << 8) | residual-in-use.  Every CTA folds all CL tags of a round, so if one
+// CTA's control flow has left the others' (a decision taken differently), every CTA sees
+// the mismatch in the same round and they all leave the walk together.
+enum AccSite : uint32_t { kSiteArgMax = 1, kSiteMaxSum = 2, kSiteSum = 3, kSiteRace = 4 };
+__device__ __forceinline__ uint32_t acc_tag(uint32_t site, int node, int cand, bool res) {
+  return (site << 24) | (static_cast<uint32_t>(node) << 16) | (static_cast<uint32_t>(cand) << 8) |
+         (res ? 1u : 0u);
+}
+
 struct AccShared {
   float4 wpart[kAccWarps];             // this CTA's warp partials
   float4 cslot[2][kAccMaxCluster];     // partial of CTA r, pushed by r (double buffered)
+  uint2 ctag[2][kAccMaxCluster];       // (tag, failed-copy flag) of CTA r's push
   uint64_t cbar[2];                    // counts the CL pushes of a round
+  uint64_t done_bar;                   // closing handshake: counts the CL "no more pushes"
   uint64_t row_bar;
   uint64_t q_bar[kAccMaxQBuf];
   int32_t par[64];
@@ -135,34 +147,39 @@ struct NoWork {
 // Cluster-wide reduction; every thread of every CTA returns the same bits.  NC components
 // are reduced over all threads; `owner(op)` is evaluated by warp 0 after the CTA's threads
 // have synchronised (so it may read what they wrote to shared memory) and folded into this
-// CTA's partial.  Each CTA pushes its partial into every peer's slot and arrives on the
-// peer's barrier; `work()` runs while the peers' partials are on their way; then each
-// warp folds the CL slots with a butterfly.
+// CTA's partial.  Each CTA pushes its partial, its `tag` and whether any of its threads saw
+// a copy fail (`failed`) into every peer's slot and arrives on the peer's barrier; `work()`
+// runs while the peers' partials are on their way; then each warp folds the CL slots with
+// a butterfly.  `bad` comes back set, the same in every thread of every CTA that got all
+// CL pushes, when the CL tags differ or a CTA flagged a failed copy; it is also set in a
+// CTA whose wait for the pushes gave up.
 template <int NC, class Op, class Owner = NoOwner, class Work = NoWork>
 __device__ __forceinline__ float4 cluster_reduce(AccShared& sh, float4 v, Op op, int& round,
-                                                 uint32_t CL, uint32_t cr, Owner owner = Owner(),
-                                                 Work work = Work()) {
+                                                 uint32_t CL, uint32_t cr, uint32_t tag, int failed,
+                                                 bool& bad, Owner owner = Owner(), Work work = Work()) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int buf = round & 1;
   v = warp_reduce_nc<NC>(v, op, 16);
   if (lane == 0) sh.wpart[warp] = v;
-  __syncthreads();
+  const int any_failed = __syncthreads_or(failed);
   if (warp == 0) {
     float4 t = lane < kAccWarps ? sh.wpart[lane] : Op::identity();
     t = op(warp_reduce_nc<NC>(t, op, kAccWarps / 2), owner(op));
     if (static_cast<uint32_t>(lane) < CL) {
       dsmem_st_f4(dsmem_map(smem_u32(&sh.cslot[buf][cr]), lane), t);
+      dsmem_st_u2(dsmem_map(smem_u32(&sh.ctag[buf][cr]), lane), make_uint2(tag, any_failed ? 1u : 0u));
       mbar_arrive_remote(dsmem_map(smem_u32(&sh.cbar[buf]), lane));
     }
   }
   work();
-  mbar_wait_cluster(smem_u32(&sh.cbar[buf]), (round >> 1) & 1, kErrAccClusterWait);
+  const bool arrived = mbar_wait_cluster(smem_u32(&sh.cbar[buf]), (round >> 1) & 1, kErrAccClusterWait);
   // lane r folds CTA r's partial; a butterfly over all 32 lanes (all four components: the
   // owner fields ride along) leaves the same bits in every lane of every warp.  Every
   // thread must get the result: the walk's control flow is decided from it, and a thread
   // that decided differently would desynchronise the CTA's barriers.
-  float4 t = static_cast<uint32_t>(lane) < CL ? sh.cslot[buf][lane & (kAccMaxCluster - 1)]
-                                              : Op::identity();
+  const int slot = static_cast<uint32_t>(lane) < CL ? lane : 0;
+  float4 t = static_cast<uint32_t>(lane) < CL ? sh.cslot[buf][slot] : Op::identity();
+  const uint2 tg = sh.ctag[buf][slot];
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     float4 o;
@@ -172,6 +189,11 @@ __device__ __forceinline__ float4 cluster_reduce(AccShared& sh, float4 v, Op op,
     o.w = __shfl_xor_sync(0xffffffffu, t.w, off);
     t = op(t, o);
   }
+  const bool mismatch = __reduce_min_sync(0xffffffffu, tg.x) != __reduce_max_sync(0xffffffffu, tg.x);
+  const bool flagged = __reduce_or_sync(0xffffffffu, tg.y) != 0u;
+  if (mismatch && threadIdx.x == 0) record_error(kErrAccDiverged);
+  // one verdict per CTA, so its threads keep to the same barriers
+  bad = __syncthreads_or(!arrived || mismatch || flagged) != 0;
   ++round;
   return t;
 }
@@ -202,16 +224,19 @@ __device__ __forceinline__ void fetch_slice(float* buf, const float* src, int n,
   }
 }
 
+// Returns false if the wait gave up (the copy is then treated as failed).
 template <bool kBulk>
-__device__ __forceinline__ void wait_slice(uint64_t* bar, uint32_t& phase, int n) {
+__device__ __forceinline__ bool wait_slice(uint64_t* bar, uint32_t& phase, int n) {
+  bool ok = true;
   if (kBulk) {
     if (n > 0) {
-      mbar_wait(smem_u32(bar), phase, kErrAccWait);
+      ok = mbar_wait(smem_u32(bar), phase, kErrAccWait);
       phase ^= 1u;
     }
   } else {
     __syncthreads();
   }
+  return ok;
 }
 
 // ln(-ln u_v) for tokens v .. v+3 of the race at `node` (v a multiple of 4).
@@ -234,6 +259,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
   const float T = prm.T;
   const size_t seq = static_cast<size_t>(b) * N;
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   float* rowbuf = acc_dyn;
   float* rbuf = acc_dyn + slice;          // [2][slice]
   float* ebuf = acc_dyn + 3 * slice;      // ln(-ln u_v) of the root's race
@@ -251,6 +277,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
   if (tid == 0) {
     mbar_init(smem_u32(&sh.cbar[0]), CL);
     mbar_init(smem_u32(&sh.cbar[1]), CL);
+    mbar_init(smem_u32(&sh.done_bar), CL);
     mbar_init(smem_u32(&sh.row_bar), 1);
     for (int q = 0; q < kAccMaxQBuf; ++q) mbar_init(smem_u32(&sh.q_bar[q]), 1);
     fence_mbar_init();
@@ -283,20 +310,39 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
   }
 
   uint32_t row_phase = 0, q_phase[kAccMaxQBuf] = {0u, 0u, 0u, 0u};
+  // bulk copies issued and not yet waited for (bit q: draft buffer q; bit 4: the row);
+  // the same in every thread, since every thread takes the same path
+  uint32_t pending = 0;
+  int failed = 0;     // a copy wait of this thread gave up
+  bool bad = false;   // the last reduction says the cluster must stop
+  bool done_sent = false;
   int round = 0;
   int cur = 0, nacc = 0, next = -1;
   const float invT = T > 0.f ? 1.0f / T : 0.f;
   // does this CTA own vocabulary entry x (and is x a real token)?
   auto owns = [&](int x) { return x >= v_lo && x < v_lo + n_loc; };
+  auto fetch_q = [&](int qb, int c) {
+    fetch_slice<kBulk>(qbuf + qb * slice, prm.draft + (seq + c) * V + v_lo, n_loc, &sh.q_bar[qb]);
+    if (kBulk && n_loc > 0) pending |= 1u << qb;
+  };
+  auto wait_q = [&](int qb) {
+    if (!kBulk || (pending >> qb) & 1u) failed |= !wait_slice<kBulk>(&sh.q_bar[qb], q_phase[qb], n_loc);
+    pending &= ~(1u << qb);
+  };
+  // this CTA will push nothing more: tell every peer (lane l of warp 0 made every push to
+  // peer l, so its arrival also releases them)
+  auto send_done = [&]() {
+    if (warp == 0 && static_cast<uint32_t>(lane) < CL)
+      mbar_arrive_remote(dsmem_map(smem_u32(&sh.done_bar), lane));
+    done_sent = true;
+  };
 
   // draft side of a node: candidate rows, p_hat_c(t_c) and the accept uniforms
   auto issue_draft = [&](int node) {
     const int c_begin = sh.child_start[node];
     const int kids = sh.child_start[node + 1] - c_begin;
     const int pre = min(kids, NQ);
-    for (int j = 0; j < pre; ++j)
-      fetch_slice<kBulk>(qbuf + j * slice, prm.draft + (seq + sh.child_list[c_begin + j]) * V + v_lo,
-                         n_loc, &sh.q_bar[j]);
+    for (int j = 0; j < pre; ++j) fetch_q(j, sh.child_list[c_begin + j]);
     if (tid < kids) {
       const int c = sh.child_list[c_begin + tid];
       sh.qx[tid] = prm.draft[(seq + c) * V + sh.tok[c]];
@@ -323,7 +369,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     const int kids = c_end - c_begin;
     if (depth > 0 && T > 0.f) issue_draft(cur);
     fetch_slice<kBulk>(rowbuf, row + v_lo, n_loc, &sh.row_bar);
-    wait_slice<kBulk>(&sh.row_bar, row_phase, n_loc);
+    failed |= !wait_slice<kBulk>(&sh.row_bar, row_phase, n_loc);
     __syncthreads();  // qx / ux visible
 
     if (T == 0.f) {
@@ -337,7 +383,9 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
           if (i + e < n_loc && xs[e] > best.x)
             best = make_float4(xs[e], __int_as_float(v_lo + i + e), 0.f, 0.f);
       }
-      const float4 r = cluster_reduce<2>(sh, best, OpArgMax(), round, CL, cr);
+      const float4 r = cluster_reduce<2>(sh, best, OpArgMax(), round, CL, cr,
+                                         acc_tag(kSiteArgMax, cur, 0, false), failed, bad);
+      if (bad) break;
       int m = __float_as_int(r.y);
       if (m < 0 || m >= V) m = 0;  // all-NaN row
       int match = -1;
@@ -378,13 +426,14 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       }
     }
     const float4 st = cluster_reduce<2>(
-        sh, ms, OpMaxSum(), round, CL, cr,
+        sh, ms, OpMaxSum(), round, CL, cr, acc_tag(kSiteMaxSum, cur, 0, false), failed, bad,
         [&](OpMaxSum) {
           float4 o = OpMaxSum::identity();
           if (owns(x0)) o.z = rowbuf[x0 - v_lo];
           return o;
         },
         NoWork());
+    if (bad) break;
     const float M = st.x, invZ = 1.0f / st.y;
     float px_next = __expf(st.z * invT - M) * invZ;  // p at the first candidate's token
 
@@ -403,8 +452,8 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       // rejected: p <- norm(max(0, p - p_hat_c)); stored unnormalised with its mass
       const int qb = j % NQ;
       float* q = qbuf + qb * slice;
-      if (!kBulk && j >= NQ) fetch_slice<kBulk>(q, prm.draft + (seq + c) * V + v_lo, n_loc, &sh.q_bar[qb]);
-      wait_slice<kBulk>(&sh.q_bar[qb], q_phase[qb], n_loc);
+      if (!kBulk && j >= NQ) fetch_q(qb, c);
+      wait_q(qb);
       const int nb = has_res ? (cb ^ 1) : cb;
       float* dst = rbuf + nb * slice;
       const float* src = rbuf + cb * slice;
@@ -432,15 +481,17 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       // the new residual there, the previous one, and the logit
       const int xn = j + 1 < kids ? sh.tok[sh.child_list[c_begin + j + 1]] : -1;
       const float4 tot = cluster_reduce<1>(sh, make_float4(part, 0.f, 0.f, 0.f), OpSum(), round, CL, cr,
-                                        [&](OpSum) {
-                                          float4 o = OpSum::identity();
-                                          if (owns(xn)) {
-                                            o.y = dst[xn - v_lo];
-                                            o.z = has_res ? src[xn - v_lo] : 0.f;
-                                            o.w = rowbuf[xn - v_lo];
-                                          }
-                                          return o;
-                                        });
+                                           acc_tag(kSiteSum, cur, j, has_res), failed, bad,
+                                           [&](OpSum) {
+                                             float4 o = OpSum::identity();
+                                             if (owns(xn)) {
+                                               o.y = dst[xn - v_lo];
+                                               o.z = has_res ? src[xn - v_lo] : 0.f;
+                                               o.w = rowbuf[xn - v_lo];
+                                             }
+                                             return o;
+                                           });
+      if (bad) break;
       if (tot.x > 0.f) {
         cb = nb;
         invZr = 1.0f / tot.x;
@@ -452,10 +503,9 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       }
       // every thread of this CTA is past its reads of buffer qb (the reduction above
       // synchronised the CTA): refill it with a later candidate's row
-      if (kBulk && j + NQ < kids)
-        fetch_slice<kBulk>(q, prm.draft + (seq + sh.child_list[c_begin + j + NQ]) * V + v_lo, n_loc,
-                           &sh.q_bar[qb]);
+      if (kBulk && j + NQ < kids) fetch_q(qb, sh.child_list[c_begin + j + NQ]);
     }
+    if (bad) break;
     if (j_acc >= 0) {
       const int c = sh.child_list[c_begin + j_acc];
       if (tid == 0) sh.acc_nodes[nacc] = c;
@@ -463,8 +513,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       // candidates [j_acc, j_acc + NQ) may still have draft-row copies in flight: land them
       // before their buffers are reused
       if (kBulk)
-        for (int j = j_acc; j < min(kids, j_acc + NQ); ++j)
-          wait_slice<kBulk>(&sh.q_bar[j % NQ], q_phase[j % NQ], n_loc);
+        for (int j = j_acc; j < min(kids, j_acc + NQ); ++j) wait_q(j % NQ);
       __syncthreads();
       cur = c;
       continue;
@@ -499,20 +548,34 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
         if (key < best.x) best = make_float4(key, __int_as_float(v_lo + i + e), 0.f, 0.f);
       }
     }
-    const float4 r = cluster_reduce<2>(sh, best, OpArgMin(), round, CL, cr);
+    // the race ends every walk at T > 0: this CTA's push is its last, so it announces that
+    // while the peers' partials are on their way
+    const float4 r = cluster_reduce<2>(sh, best, OpArgMin(), round, CL, cr,
+                                       acc_tag(kSiteRace, cur, 0, has_res), failed, bad, NoOwner(),
+                                       send_done);
+    if (bad) break;
     next = __float_as_int(r.y);
     if (next < 0 || next >= V) next = 0;
     break;
   }
 
   if (cr == 0 && tid == 0) {
-    for (int i = 0; i < N; ++i) prm.accepted_nodes[seq + i] = i < nacc ? sh.acc_nodes[i] : -1;
-    prm.accept_len[b] = nacc;
-    prm.next_token[b] = next;
+    // a walk the cluster stopped (its CTAs disagreed, or a wait gave up) reports like an
+    // invalid tree; the device error word says why
+    for (int i = 0; i < N; ++i) prm.accepted_nodes[seq + i] = (!bad && i < nacc) ? sh.acc_nodes[i] : -1;
+    prm.accept_len[b] = bad ? -1 : nacc;
+    prm.next_token[b] = bad ? -1 : next;
   }
-  // Every CTA takes the same reductions, and a CTA's last one waited for every peer's push
-  // into its shared memory (peers only push, they never load from it), so no peer can still
-  // touch this CTA's shared memory: no closing cluster barrier is needed.
+  // Closing handshake.  A CTA leaves only once every peer has said it will push nothing
+  // more, so no push can reach the shared memory of a CTA that has exited, even if the
+  // cluster's control flow split (the tags make every CTA stop in the round after a split;
+  // a CTA that stopped on its own waits here for the others' rounds to give up).  The wait
+  // is twice as long as a reduction's, so a peer that timed out in its round still arrives
+  // in time.  Copies this CTA issued and did not consume land first.
+  if (!done_sent) send_done();
+  for (int qb = 0; qb < kAccMaxQBuf; ++qb)
+    if ((pending >> qb) & 1u) wait_q(qb);
+  if (tid == 0) mbar_wait_cluster(smem_u32(&sh.done_bar), 0, kErrAccClusterWait, 2 * kWaitLimitNs);
 }
 
 }  // namespace eagle

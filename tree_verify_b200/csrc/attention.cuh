@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(128)
     m = mn;
   };
   int L = prefix_lens[b];
+  if ((L < 0 || L > Lmax) && threadIdx.x == 0) record_error(kErrAttnPrefixLen);
   L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
   const size_t pbase = (static_cast<size_t>(b) * Hkv + g) * Lmax;
   for (int j = 0; j < L; ++j) visit(kp + (pbase + j) * D, vp + (pbase + j) * D);

@@ -34,6 +34,8 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 eagle_status_t check_shape(const eagle_shape_t* s) {
   if (s == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
   if (s->batch < 1 || s->batch > 65535) return EAGLE_ERR_INVALID_ARGUMENT;
+  // N <= 64 also keeps node indices inside the Philox counter's 8-bit node field
+  static_assert(64 - 1 <= kPhiloxMaxField, "tree nodes must fit the counter's node field");
   if (s->num_nodes < 1 || s->num_nodes > 64) return EAGLE_ERR_INVALID_ARGUMENT;
   if (s->num_q_heads < 1 || s->num_kv_heads < 1 || s->num_q_heads % s->num_kv_heads != 0)
     return EAGLE_ERR_INVALID_ARGUMENT;
@@ -91,11 +93,24 @@ AttnPlan plan_attention(const eagle_shape_t* s, bool lite = false) {
     p.ml_bytes = align256(rows * p.splits * 2 * sizeof(float));
     return p;
   }
+  // one CTA per SM at a time: pick the split count that minimises waves x (tiles per split
+  // + a CTA's fixed cost, about four tiles' time: set-up, pipeline fill, the tree tile, the
+  // partials it writes for the merge)
   const long base = static_cast<long>(s->batch) * s->num_kv_heads * p.row_blocks;
-  const long want = (static_cast<long>(kNumSMs) + base - 1) / base;
-  int tiles_per = static_cast<int>((max_tiles + want - 1) / want);
+  int best_splits = 1;
+  long best_cost = -1;
+  for (int sp = 1; sp <= (max_tiles > 0 ? max_tiles : 1); ++sp) {
+    const long tiles_per = max_tiles > 0 ? (max_tiles + sp - 1) / sp : 0;
+    if (sp > 1 && (tiles_per - 1) * sp >= max_tiles) continue;  // same split count as a smaller sp
+    const long waves = (base * sp + kNumSMs - 1) / kNumSMs;
+    const long cost = waves * (tiles_per + 4);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_splits = sp;
+    }
+  }
+  int tiles_per = max_tiles > 0 ? (max_tiles + best_splits - 1) / best_splits : 1;
   if (tiles_per < 1) tiles_per = 1;
-  if (tiles_per > 32) tiles_per = 32;
   p.tiles_per_split = tiles_per;
   p.splits = max_tiles > 0 ? (max_tiles + tiles_per - 1) / tiles_per : 1;
   if (s->dtype != EAGLE_DTYPE_BF16 || p.splits == 1) {
@@ -223,7 +238,7 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t*
                  const cuuint64_t* strides, const cuuint32_t* box) {
   auto enc = get_encode();
   if (enc == nullptr) return false;
-  cuuint32_t es[3] = {1, 1, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
   const CUresult r =
       enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
           dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -264,6 +279,10 @@ bool ensure_attributes(int dev) {
   std::call_once(st.attrs_once, [&] {
     bool ok = true;
     ok &= cudaFuncSetAttribute(lm_head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(lm_head_tc_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(lm_head_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TcSmem<64>::kAlloc) == cudaSuccess;
@@ -347,7 +366,7 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   }
   const AttnPlan plan = plan_attention(s, lite);
   const int G = Hq / Hkv;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tkt, tvt;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax),
                               static_cast<cuuint64_t>(B) * Hkv};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Lmax) * D * 2};
@@ -357,8 +376,16 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
                                static_cast<cuuint64_t>(B) * s->num_nodes};
   const cuuint64_t qstrides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hq) * D * 2};
   const cuuint32_t qbox[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(plan.nodes_per_block)};
+  // tree K/V viewed as [B][N][Hkv][D]: one box = the 64 node rows of (b, kv head), rows
+  // past N outside the tensor (zero-filled)
+  const cuuint64_t tdims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
+                               static_cast<cuuint64_t>(s->num_nodes), static_cast<cuuint64_t>(B)};
+  const cuuint64_t tstrides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hkv) * D * 2,
+                                  static_cast<cuuint64_t>(s->num_nodes) * Hkv * D * 2};
+  const cuuint32_t tbox[4] = {64, 1, static_cast<cuuint32_t>(kAttnKeys), 1};
   if (!encode_bf16(&tk, kp, 3, dims, strides, box) || !encode_bf16(&tv, vp, 3, dims, strides, box) ||
-      !encode_bf16(&tq, q, 3, qdims, qstrides, qbox))
+      !encode_bf16(&tq, q, 3, qdims, qstrides, qbox) || !encode_bf16(&tkt, kt, 4, tdims, tstrides, tbox) ||
+      !encode_bf16(&tvt, vt, 4, tdims, tstrides, tbox))
     return EAGLE_ERR_CUDA;
   TcAttnParams tp{};
   AttnParams& prm = tp.a;
@@ -388,11 +415,11 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   cfg.stream = st;
   cudaError_t e;
   if (plan.lite)
-    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64, true>, tq, tk, tv, tp)
-                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128, true>, tq, tk, tv, tp);
+    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64, true>, tq, tk, tv, tkt, tvt, tp)
+                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128, true>, tq, tk, tv, tkt, tvt, tp);
   else
-    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, tq, tk, tv, tp)
-                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, tq, tk, tv, tp);
+    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, tq, tk, tv, tkt, tvt, tp)
+                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, tq, tk, tv, tkt, tvt, tp);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EAGLE_ERR_CUDA;
@@ -408,6 +435,83 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   return launch_status();
 }
 
+// Many tree rows (more than one chunk of 256): the persistent kernel, one CTA per SM, the
+// chunks of a vocabulary tile on neighbouring CTAs, the epilogue of one tile under the
+// MMAs of the next.
+eagle_status_t run_lm_head_persistent(const eagle_shape_t* s, const void* hidden, const void* w,
+                                      float* logits, cudaStream_t st, const LmPlan& plan) {
+  const int M = s->batch * s->num_nodes, V = s->vocab, H = s->hidden;
+  CUtensorMap tw, th;
+  const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
+  const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};
+  const cuuint64_t stride[1] = {static_cast<cuuint64_t>(H) * 2};
+  const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(kLmBlockV)};
+  const cuuint32_t hbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(plan.bn)};
+  if (!encode_bf16(&tw, w, 2, wd, stride, wbox) || !encode_bf16(&th, hidden, 2, hd, stride, hbox))
+    return EAGLE_ERR_CUDA;
+  const int vtiles = (V + kLmBlockV - 1) / kLmBlockV;
+  // hidden boxes mostly hit L2: a short ring; W boxes come from HBM: the rest of the
+  // shared memory, so they are issued several k-blocks ahead
+  const int hstages = kLmpHiddenStages;
+  int wstages = 2;
+  while (wstages < kLmpMaxStages && lmp_smem_bytes(plan.bn, wstages + 1, hstages) <= 220 * 1024) ++wstages;
+  LmpParams prm{logits, M, V, H, plan.bn, plan.chunks, vtiles, wstages, hstages};
+  const size_t smem = lmp_smem_bytes(plan.bn, wstages, hstages);
+  const long tiles = static_cast<long>(vtiles) * plan.chunks;
+  const int grid = static_cast<int>(tiles < kNumSMs ? tiles : kNumSMs);
+  lm_head_tc_persist_kernel<<<grid, kLmpThreads, smem, st>>>(tw, th, prm);
+  return launch_status();
+}
+
+// The CTA-pair kernel: tree rows in chunks of a multiple of 32 (each CTA of a pair holds
+// half of a chunk), picked to waste the fewest padded rows.
+eagle_status_t run_lm_head_pair(const eagle_shape_t* s, const void* hidden, const void* w,
+                                float* logits, cudaStream_t st) {
+  const int M = s->batch * s->num_nodes, V = s->vocab, H = s->hidden;
+  int chunks = (M + 255) / 256, bn = 0;
+  long best = -1;
+  for (int c = chunks; c <= chunks + 2; ++c) {
+    const int b = ((M + c - 1) / c + 31) / 32 * 32;
+    if (b > 256) continue;
+    if (best < 0 || static_cast<long>(c) * b < best) {
+      best = static_cast<long>(c) * b;
+      chunks = c;
+      bn = b;
+    }
+  }
+  CUtensorMap tw, th;
+  const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
+  const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};
+  const cuuint64_t stride[1] = {static_cast<cuuint64_t>(H) * 2};
+  const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(kLmBlockV)};
+  const cuuint32_t hbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(bn / 2)};
+  if (!encode_bf16(&tw, w, 2, wd, stride, wbox) || !encode_bf16(&th, hidden, 2, hd, stride, hbox))
+    return EAGLE_ERR_CUDA;
+  const int vpairs = (V + 2 * kLmBlockV - 1) / (2 * kLmBlockV);
+  int stages = 2;
+  while (stages < 12 && lm2_smem_bytes(bn, stages + 1) <= 220 * 1024) ++stages;
+  Lm2Params prm{logits, M, V, H, bn, chunks, vpairs, stages};
+  const long tiles = static_cast<long>(vpairs) * chunks;
+  const int pairs = static_cast<int>(tiles < kNumSMs / 2 ? tiles : kNumSMs / 2);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kLm2Threads);
+  cfg.dynamicSmemBytes = lm2_smem_bytes(bn, stages);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, lm_head_tc_pair_kernel, tw, th, prm) != cudaSuccess) {
+    cudaGetLastError();
+    return EAGLE_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // `started`: an event that fires once every CTA has begun (the LM head's resources are
 // claimed), for a second stream to start work beside it; `max_stages` caps the TMA ring.
 eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const void* w, float* logits,
@@ -420,6 +524,11 @@ eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const voi
     return launch_status();
   }
   const LmPlan plan = plan_lm_head(s, max_stages);
+#ifdef EAGLE_LM_PAIR
+  if (plan.chunks > 1 && started == nullptr) return run_lm_head_pair(s, hidden, w, logits, st);
+#else
+  if (plan.chunks > 1 && started == nullptr) return run_lm_head_persistent(s, hidden, w, logits, st, plan);
+#endif
   CUtensorMap tw, th;
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
   const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};
@@ -684,6 +793,9 @@ eagle_status_t draft_launch(int mode, int32_t batch, int32_t rows_per_seq, int32
   if (batch < 1 || batch > 65535 || rows_per_seq < 1 || rows_per_seq > 256 || k < 1 ||
       k > kDraftMaxK || vocab < k)
     return EAGLE_ERR_INVALID_ARGUMENT;
+  // the Philox counter packs b (16 bits), the purpose 2 + j and the row f (8 bits each)
+  static_assert(kDraftMaxK + 2 <= 256, "race purposes must fit the counter's 8-bit field");
+  if (rows_per_seq - 1 > kPhiloxMaxField || k + 1 > kPhiloxMaxField) return EAGLE_ERR_INVALID_ARGUMENT;
   if (!(temperature >= 0.f) || !std::isfinite(temperature)) return EAGLE_ERR_INVALID_ARGUMENT;
   if (logits == nullptr || tokens == nullptr || conf == nullptr) return EAGLE_ERR_INVALID_ARGUMENT;
   if ((reinterpret_cast<uintptr_t>(logits) & 3) != 0) return EAGLE_ERR_INVALID_ARGUMENT;
@@ -941,20 +1053,23 @@ namespace {
 static __device__ __align__(256) uint8_t g_static_scratch[EAGLE_STATIC_SCRATCH_BYTES];
 
 struct StaticScratch {
-  std::once_flag once;
-  cudaError_t status = cudaErrorUnknown;
-  void* ptr = nullptr;
+  std::mutex mu;
+  void* ptr = nullptr;  // set only by a lookup that succeeded
 };
 StaticScratch g_scratch[kMaxDevices];
 
-// The host-side name of the array is not a device address; look the address up once per
-// device, with that device current.
+// The host-side name of the array is not a device address; look the address up per
+// device, with that device current.  Only a successful lookup is kept: one that failed
+// (say, made during a stream capture) is retried by the next call.
 void* static_scratch_address(int dev) {
   StaticScratch& s = g_scratch[dev];
-  std::call_once(s.once, [&] {
-    s.status = cudaGetSymbolAddress(&s.ptr, g_static_scratch);
-  });
-  return s.status == cudaSuccess ? s.ptr : nullptr;
+  std::lock_guard<std::mutex> lock(s.mu);
+  if (s.ptr == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) == cudaSuccess) s.ptr = p;
+    else cudaGetLastError();
+  }
+  return s.ptr;
 }
 
 }  // namespace

@@ -13,6 +13,10 @@
 
 namespace eagle {
 
+// b fills 16 bits of the counter word, purpose and node 8 bits each: callers keep
+// node, purpose <= kPhiloxMaxField and b <= 65535 (checked on the host).
+constexpr int kPhiloxMaxField = 255;
+
 struct Philox4 {
   uint32_t w[4];
 };

@@ -66,7 +66,8 @@ def test_static_scratch_matches_workspace_entry_point(cuda_lib):
 
 def test_static_scratch_rejects_shapes_beyond_its_size(cuda_lib):
     fn = _static_fn(cuda_lib)
-    shape = cuda_lib.make_shape(8, 64, 32, 8, 128, 8192, 64, 128, "bf16")
+    # 2 sequences, 64 query / 8 kv heads, a 64K-token prefix: split partials of ~37 MB
+    shape = cuda_lib.make_shape(2, 64, 64, 8, 128, 65536, 64, 128, "bf16")
     assert cuda_lib.workspace_bytes(shape) > STATIC_SCRATCH_BYTES
     fake = 1 << 20
     rc = fn(ctypes.byref(shape), *([fake] * 8), None)

@@ -11,7 +11,8 @@
 //     children's draft rows come into shared memory at once by bulk async copies (one
 //     mbarrier per buffer); p_hat_c(t_c) and the accept uniforms are fetched or computed
 //     in the same round trip, so each later pass over V reads shared memory; the root's
-//     race keys (ln(-ln u_v)) are computed before the logits are awaited;
+//     race keys (ln(-ln u_v)) are computed before the logits are awaited, those of every
+//     later node while its first reduction waits for the peers;
 //   - the root's draft rows are fetched before waiting for the LM-head grid (programmatic
 //     dependent launch), so they arrive while the logits are still being produced;
 //   - the residual r = max(0, p - p_hat) stays in the owners' shared memory (two buffers,
@@ -19,8 +20,10 @@
 //     test needs (r[t], logits[t]) ride along with the reduction that precedes it;
 //   - every reduction (max / sum-exp, argmax, sum, race argmin) is a warp butterfly, a
 //     combine of the CTA's warps, and a push of the CTA's partial into every peer's shared
-//     memory with a remote mbarrier arrival; each CTA then combines the CL partials in rank
-//     order, so all CTAs reach bit-identical decisions without a cluster-wide barrier.
+//     memory with a remote mbarrier arrival; each CTA then folds the CL partials with a
+//     butterfly, so all CTAs reach bit-identical decisions without a cluster-wide barrier;
+//     the max / sum-exp statistics combine in two passes at each level (the maximum, then
+//     one exponential per partial and a sum), which keeps the dependent chain short.
 // Only the accepted node indices, their count and the one extra token are written.
 #pragma once
 
@@ -53,22 +56,10 @@ struct AccParams {
 
 // ---------------------------------------------------------------- reduction operators
 // Payload float4.  Every operator is commutative bit for bit, so a butterfly leaves all
-// lanes equal.  Components .z/.w of OpMaxSum and .y/.z/.w of OpSum are "owner fields":
-// exactly one CTA contributes a nonzero value (a scalar it alone holds in shared memory)
-// and the others contribute 0, so adding them broadcasts that scalar exactly.
-struct OpMaxSum {  // (max y, sum exp(y - max), owner fields)
-  static __device__ __forceinline__ float4 identity() { return make_float4(-INFINITY, 0.f, 0.f, 0.f); }
-  __device__ __forceinline__ float4 operator()(float4 a, float4 b) const {
-    const float m = fmaxf(a.x, b.x);
-    // each product rounded on its own: a contracted a*x + b*y (one product fused into the
-    // add) rounds differently from b*y + a*x, and lanes holding op(a, b) and op(b, a)
-    // would then disagree on Z
-    const float s = m == -INFINITY
-                        ? 0.f
-                        : __fadd_rn(__fmul_rn(a.y, __expf(a.x - m)), __fmul_rn(b.y, __expf(b.x - m)));
-    return make_float4(m, s, a.z + b.z, a.w + b.w);
-  }
-};
+// lanes equal.  Components .y/.z/.w of OpSum (and .z of the max / sum-exp reduction) are
+// "owner fields": exactly one CTA contributes a nonzero value (a scalar it alone holds in
+// shared memory) and the others contribute 0, so adding them broadcasts that scalar
+// exactly.
 struct OpArgMax {  // (value, index bits): larger value, then lower index
   static __device__ __forceinline__ float4 identity() {
     return make_float4(-INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
@@ -198,6 +189,67 @@ __device__ __forceinline__ float4 cluster_reduce(AccShared& sh, float4 v, Op op,
   return t;
 }
 
+// Cluster-wide (max y, sum exp(y - max)) of the row's statistics, with the same push /
+// tag / wait protocol as cluster_reduce.  Each level combines in two passes -- the maximum
+// by a butterfly, then every partial rescaled to it with one exponential and summed by a
+// butterfly -- instead of merging pairs with two exponentials per step, so the dependent
+// chain of exponentials is one per level.  Every thread of every CTA returns the same bits
+// (fmaxf and fp32 addition are commutative bit for bit).  (m, s): this thread's partial,
+// s taken relative to m.  `owner_z`: warp 0's contribution to the owner field .z.
+template <class Work = NoWork>
+__device__ __forceinline__ float4 cluster_maxsum(AccShared& sh, float m, float s, int& round, uint32_t CL,
+                                                 uint32_t cr, uint32_t tag, int failed, bool& bad,
+                                                 float owner_z, Work work = Work()) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int buf = round & 1;
+  // warp: max, then rescale and sum
+  float wm = m;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, off));
+  float ws = wm == -INFINITY ? 0.f : s * __expf(m - wm);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
+  if (lane == 0) sh.wpart[warp] = make_float4(wm, ws, 0.f, 0.f);
+  const int any_failed = __syncthreads_or(failed);
+  if (warp == 0) {
+    const float4 p = lane < kAccWarps ? sh.wpart[lane] : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    float cm = p.x;
+#pragma unroll
+    for (int off = kAccWarps / 2; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+    float cs = cm == -INFINITY ? 0.f : p.y * __expf(p.x - cm);
+#pragma unroll
+    for (int off = kAccWarps / 2; off > 0; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
+    const float4 t = make_float4(cm, cs, owner_z, 0.f);
+    if (static_cast<uint32_t>(lane) < CL) {
+      dsmem_st_f4(dsmem_map(smem_u32(&sh.cslot[buf][cr]), lane), t);
+      dsmem_st_u2(dsmem_map(smem_u32(&sh.ctag[buf][cr]), lane), make_uint2(tag, any_failed ? 1u : 0u));
+      mbar_arrive_remote(dsmem_map(smem_u32(&sh.cbar[buf]), lane));
+    }
+  }
+  work();
+  const bool arrived = mbar_wait_cluster(smem_u32(&sh.cbar[buf]), (round >> 1) & 1, kErrAccClusterWait);
+  const int slot = static_cast<uint32_t>(lane) < CL ? lane : 0;
+  const float4 p = static_cast<uint32_t>(lane) < CL ? sh.cslot[buf][slot] : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+  const uint2 tg = sh.ctag[buf][slot];
+  float M = p.x;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float Z = M == -INFINITY ? 0.f : p.y * __expf(p.x - M);
+  float z = p.z, wv = p.w;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    Z += __shfl_xor_sync(0xffffffffu, Z, off);
+    z += __shfl_xor_sync(0xffffffffu, z, off);
+    wv += __shfl_xor_sync(0xffffffffu, wv, off);
+  }
+  const bool mismatch = __reduce_min_sync(0xffffffffu, tg.x) != __reduce_max_sync(0xffffffffu, tg.x);
+  const bool flagged = __reduce_or_sync(0xffffffffu, tg.y) != 0u;
+  if (mismatch && threadIdx.x == 0) record_error(kErrAccDiverged);
+  bad = __syncthreads_or(!arrived || mismatch || flagged) != 0;
+  ++round;
+  return make_float4(M, Z, z, wv);
+}
+
 // Bulk async copy of `bytes` (multiple of 16, both ends 16-byte aligned) into shared memory,
 // completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -239,11 +291,13 @@ __device__ __forceinline__ bool wait_slice(uint64_t* bar, uint32_t& phase, int n
   return ok;
 }
 
-// ln(-ln u_v) for tokens v .. v+3 of the race at `node` (v a multiple of 4).
+// ln(-ln u_v) for tokens v .. v+3 of the race at `node` (v a multiple of 4).  The inner
+// logarithm is the accurate one (for u near 1, -ln u is tiny and a fast logarithm's absolute
+// error would be a large relative one); the outer one only needs a small absolute error.
 __device__ __forceinline__ float4 race_keys(uint64_t seed, uint64_t offset, int b, int node, int v) {
   const Philox4 rnd = philox_group(seed, offset, b, node, 1, static_cast<uint32_t>(v) >> 2);
-  return make_float4(logf(-logf(word_to_uniform(rnd.w[0]))), logf(-logf(word_to_uniform(rnd.w[1]))),
-                     logf(-logf(word_to_uniform(rnd.w[2]))), logf(-logf(word_to_uniform(rnd.w[3]))));
+  return make_float4(__logf(-logf(word_to_uniform(rnd.w[0]))), __logf(-logf(word_to_uniform(rnd.w[1]))),
+                     __logf(-logf(word_to_uniform(rnd.w[2]))), __logf(-logf(word_to_uniform(rnd.w[3]))));
 }
 
 template <bool kBulk>
@@ -262,7 +316,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
   const int warp = tid >> 5, lane = tid & 31;
   float* rowbuf = acc_dyn;
   float* rbuf = acc_dyn + slice;          // [2][slice]
-  float* ebuf = acc_dyn + 3 * slice;      // ln(-ln u_v) of the root's race
+  float* ebuf = acc_dyn + 3 * slice;      // ln(-ln u_v) of one node's race
   float* qbuf = acc_dyn + 4 * slice;      // [NQ][slice]
 
   // ---- tree set-up (inputs only; runs while the LM-head grid may still be running)
@@ -349,12 +403,17 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       sh.ux[tid] = uniform_at(prm.seed, prm.offset, b, c, 0, 0);
     }
   };
+  // ebuf holds the race keys of node `ekey`: the root's, computed now (the walk most often
+  // ends there), later those of each visited node, computed while its first reduction
+  // waits for the peers; each thread keeps the keys of the entries it later races over
+  int ekey = 0;
+  auto fill_keys = [&](int node) {
+    for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads)
+      *reinterpret_cast<float4*>(ebuf + i) = race_keys(prm.seed, prm.offset, b, node, v_lo + i);
+  };
   if (T > 0.f) {
     issue_draft(0);
-    // the root's race keys (the walk most often ends there); each thread keeps the keys of
-    // the entries it later races over
-    for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads)
-      *reinterpret_cast<float4*>(ebuf + i) = race_keys(prm.seed, prm.offset, b, 0, v_lo + i);
+    fill_keys(0);
   }
 
   // the logits come from the LM-head grid launched just before this one
@@ -367,8 +426,9 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     const float* row = prm.logits + (seq + cur) * V;
     const int c_begin = sh.child_start[cur], c_end = sh.child_start[cur + 1];
     const int kids = c_end - c_begin;
-    if (depth > 0 && T > 0.f) issue_draft(cur);
+    // the row's copy first, so the draft side's loads overlap it
     fetch_slice<kBulk>(rowbuf, row + v_lo, n_loc, &sh.row_bar);
+    if (depth > 0 && T > 0.f) issue_draft(cur);
     failed |= !wait_slice<kBulk>(&sh.row_bar, row_phase, n_loc);
     __syncthreads();  // qx / ux visible
 
@@ -406,33 +466,37 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       break;
     }
 
-    // p = softmax(logits[cur] / T): statistics (M, Z) of y = l / T; the owner of the first
-    // candidate's token also broadcasts its logit
+    // p = softmax(logits[cur] / T): statistics (M, Z) of y = l / T, in two passes over the
+    // slice (the maximum, then the exponentials: independent operations, no chain); the
+    // owner of the first candidate's token also broadcasts its logit
     const int x0 = kids > 0 ? sh.tok[sh.child_list[c_begin]] : -1;
-    float4 ms = OpMaxSum::identity();
+    float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
       const float4 x = *reinterpret_cast<const float4*>(rowbuf + i);
-      const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (i + e >= n_loc) break;
-        const float y = xs[e] * invT;
-        if (y > ms.x) {
-          ms.y = ms.y * __expf(ms.x - y) + 1.f;
-          ms.x = y;
-        } else {
-          ms.y += __expf(y - ms.x);
-        }
+      mq[0] = fmaxf(mq[0], x.x);
+      if (i + 1 < n_loc) mq[1] = fmaxf(mq[1], x.y);
+      if (i + 2 < n_loc) mq[2] = fmaxf(mq[2], x.z);
+      if (i + 3 < n_loc) mq[3] = fmaxf(mq[3], x.w);
+    }
+    const float mt = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * invT;
+    float sq[4] = {0.f, 0.f, 0.f, 0.f};
+    if (mt != -INFINITY) {
+      for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
+        const float4 x = *reinterpret_cast<const float4*>(rowbuf + i);
+        sq[0] += __expf(x.x * invT - mt);
+        if (i + 1 < n_loc) sq[1] += __expf(x.y * invT - mt);
+        if (i + 2 < n_loc) sq[2] += __expf(x.z * invT - mt);
+        if (i + 3 < n_loc) sq[3] += __expf(x.w * invT - mt);
       }
     }
-    const float4 st = cluster_reduce<2>(
-        sh, ms, OpMaxSum(), round, CL, cr, acc_tag(kSiteMaxSum, cur, 0, false), failed, bad,
-        [&](OpMaxSum) {
-          float4 o = OpMaxSum::identity();
-          if (owns(x0)) o.z = rowbuf[x0 - v_lo];
-          return o;
-        },
-        NoWork());
+    const float st_own = owns(x0) ? rowbuf[x0 - v_lo] : 0.f;
+    const bool new_keys = ekey != cur;
+    const float4 st = cluster_maxsum(sh, mt, (sq[0] + sq[1]) + (sq[2] + sq[3]), round, CL, cr,
+                                     acc_tag(kSiteMaxSum, cur, 0, false), failed, bad, st_own, [&]() {
+                                       // this node's race keys, in case the walk ends here
+                                       if (new_keys) fill_keys(cur);
+                                     });
+    ekey = cur;
     if (bad) break;
     const float M = st.x, invZ = 1.0f / st.y;
     float px_next = __expf(st.z * invT - M) * invZ;  // p at the first candidate's token
@@ -524,8 +588,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     float4 best = OpArgMin::identity();
     const float* src = rbuf + cb * slice;
     for (int i = 4 * tid; i < n_loc; i += 4 * kAccThreads) {
-      const float4 e4 = cur == 0 ? *reinterpret_cast<const float4*>(ebuf + i)
-                                 : race_keys(prm.seed, prm.offset, b, cur, v_lo + i);
+      const float4 e4 = *reinterpret_cast<const float4*>(ebuf + i);  // keys of node cur
       const float es[4] = {e4.x, e4.y, e4.z, e4.w};
       float lw[4];
       if (has_res) {

@@ -105,6 +105,11 @@ __global__ void __launch_bounds__(128)
 }
 
 // ------------------------------------------------------------------ fp32 path
+// One warp per output row.  Keys go 32 at a time: lane j scores key c + j against the row's
+// query (kept in shared memory, read as a broadcast), the warp folds the 32 scores into
+// the running maximum and denominator, then every lane accumulates its D/32 output
+// columns over those keys (coalesced V rows).  The loads of a chunk are independent of
+// one another, so a row costs a few memory round trips per 32 keys rather than one per key.
 
 template <int D>
 __global__ void __launch_bounds__(128)
@@ -113,7 +118,10 @@ __global__ void __launch_bounds__(128)
                          const float* __restrict__ kt, const float* __restrict__ vt,
                          const int32_t* __restrict__ parents, float* __restrict__ out, int B, int N,
                          int Hq, int Hkv, int Lmax, float scale) {
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  __shared__ float q_s[4][D];
+  __shared__ int path_s[4][64];
+  const int wid = threadIdx.x >> 5;
+  const int row = blockIdx.x * 4 + wid;
   const int lane = threadIdx.x & 31;
   if (row >= B * N * Hq) return;
   const int b = row / (N * Hq);
@@ -121,40 +129,67 @@ __global__ void __launch_bounds__(128)
   const int h = row % Hq;
   const int g = h / (Hq / Hkv);
   constexpr int kPer = D / 32;
-  float qv[kPer], acc[kPer];
+  float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    qv[e] = q[static_cast<size_t>(row) * D + lane + 32 * e];
+    q_s[wid][lane + 32 * e] = q[static_cast<size_t>(row) * D + lane + 32 * e];
     acc[e] = 0.f;
   }
-  float m = -INFINITY, l = 0.f;
-  auto visit = [&](const float* kr, const float* vr) {
-    float s = 0.f;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) s = fmaf(qv[e], kr[lane + 32 * e], s);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    s *= scale;
-    const float mn = fmaxf(m, s);
-    const float corr = expf(m - mn);
-    const float p = expf(s - mn);
-    l = l * corr + p;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[e] = fmaf(p, vr[lane + 32 * e], acc[e] * corr);
-    m = mn;
-  };
+  // the node's path to the root (a link that does not point to an earlier node ends it)
+  int np = 0;
+  if (lane == 0) {
+    int a = i;
+    for (int guard = 0; guard < 64 && a >= 0; ++guard) {
+      path_s[wid][np++] = a;
+      const int p = parents[static_cast<size_t>(b) * N + a];
+      a = (p >= 0 && p < a) ? p : -1;
+    }
+  }
+  np = __shfl_sync(0xffffffffu, np, 0);
+  __syncwarp();
   int L = prefix_lens[b];
-  if ((L < 0 || L > Lmax) && threadIdx.x == 0) record_error(kErrAttnPrefixLen);
+  if ((L < 0 || L > Lmax) && lane == 0) record_error(kErrAttnPrefixLen);
   L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
   const size_t pbase = (static_cast<size_t>(b) * Hkv + g) * Lmax;
-  for (int j = 0; j < L; ++j) visit(kp + (pbase + j) * D, vp + (pbase + j) * D);
-  int a = i;
-  for (;;) {
-    const size_t off = ((static_cast<size_t>(b) * N + a) * Hkv + g) * D;
-    visit(kt + off, vt + off);
-    const int p = parents[static_cast<size_t>(b) * N + a];
-    if (p < 0 || p >= a) break;
-    a = p;
+  auto key_row = [&](int j, const float* pre, const float* tree) -> const float* {
+    return j < L ? pre + (pbase + j) * D
+                 : tree + ((static_cast<size_t>(b) * N + path_s[wid][j - L]) * Hkv + g) * D;
+  };
+  const int nk = L + np;
+  float m = -INFINITY, l = 0.f;
+  for (int c = 0; c < nk; c += 32) {
+    const int j = c + lane;
+    float s = -INFINITY;
+    if (j < nk) {
+      const float* kr = key_row(j, kp, kt);
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll 8
+      for (int d = 0; d < D; d += 2) {
+        d0 = fmaf(q_s[wid][d], kr[d], d0);
+        d1 = fmaf(q_s[wid][d + 1], kr[d + 1], d1);
+      }
+      s = (d0 + d1) * scale;
+    }
+    float cm = s;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+    const float mn = fmaxf(m, cm);
+    const float corr = expf(m - mn);
+    const float p = j < nk ? expf(s - mn) : 0.f;
+    float ps = p;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+    l = l * corr + ps;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] *= corr;
+    const int cnt = min(32, nk - c);
+    for (int t = 0; t < cnt; ++t) {
+      const float pt = __shfl_sync(0xffffffffu, p, t);
+      const float* vr = key_row(c + t, vp, vt);
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] = fmaf(pt, vr[lane + 32 * e], acc[e]);
+    }
+    m = mn;
   }
   const float inv = 1.0f / l;
 #pragma unroll

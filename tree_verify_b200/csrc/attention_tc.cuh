@@ -7,21 +7,22 @@
 // r -> node i0 + r / G, head kvh*G + r % G), so one 128-row MMA tile covers all of them and
 // every prefix K/V tile is read from HBM once.
 //
-//   warp 8 (lane 0)   TMA: the Q tile once (a 3-D box over [B*N, Hq, D]) and the 64-key K
+//   warp 16 (lane 0)  TMA: the Q tile once (a 3-D box over [B*N, Hq, D]) and the 64-key K
 //                     tiles of this split into the K ring;
-//   warp 10 (lane 0)  TMA: the matching V tiles into the V ring (its own ring and barriers,
+//   warp 18 (lane 0)  TMA: the matching V tiles into the V ring (its own ring and barriers,
 //                     so a K slot is refilled as soon as S = Q K^T has read it, a tile
 //                     earlier than its V slot);
-//   warp 9 (lane 0)   tcgen05.mma: S = Q K^T (M 128, N 64, K = D) into one of two TMEM
+//   warp 17 (lane 0)  tcgen05.mma: S = Q K^T (M 128, N 64, K = D) into one of two TMEM
 //                     buffers, then O += P V (M 128, N = D, K 64) with P read from TMEM and
 //                     V as an MN-major operand straight from its TMA tile;
-//   warps 0-7         two threads per query row (= TMEM lane): warps w and w + 4 share the
-//                     lane quarter w and take 32 of the tile's 64 scores each (tcgen05.ld),
-//                     mask them (prefix length, or the ancestor bitmask for the tree tile),
-//                     exchange the row maximum through shared memory, and store their half
-//                     of P (bf16 pairs) back into TMEM (tcgen05.st).  A warp whose 32 rows
-//                     are all padding (fewer than 128 query rows) only keeps the barriers.
-// S(t+1) is computed while the softmax of tile t runs.  O lives in TMEM and is rescaled
+//   warps 0-15        four threads per query row (= TMEM lane): warps w, w + 4, w + 8 and
+//                     w + 12 share the lane quarter w % 4 and take 16 of the tile's 64 scores
+//                     each (tcgen05.ld), mask them (prefix length, or the ancestor bitmask
+//                     for the tree tile), exchange the row maximum through shared memory,
+//                     and store their quarter of P (bf16 pairs) back into TMEM (tcgen05.st).
+//                     Four warps per SM sub-partition keep the exponential unit fed.  A
+//                     warp whose 32 rows are all padding only keeps the barriers.
+// S(t+1) and S(t+2) are computed while the softmax of tile t runs (three S and P buffers).  O lives in TMEM and is rescaled
 // lazily: only when a row's maximum grows by more than 2^8 over the reference the row's P
 // values were taken against (otherwise P <= 2^8, well inside bf16/fp32 range).  The last
 // split also runs the tree tile: its K/V rows come by TMA from a 4-D view of the tree K/V
@@ -35,7 +36,9 @@
 namespace eagle {
 
 constexpr int kTcRows = 128;  // MMA M: query rows per CTA
-constexpr int kTcSoftmaxWarps = 8;
+constexpr int kTcSoftmaxWarps = 16;
+constexpr int kTcParts = kTcSoftmaxWarps / 4;       // warps sharing one TMEM lane quarter
+constexpr int kTcCols = 64 / kTcParts;              // score columns per softmax thread
 constexpr int kTcKWarp = kTcSoftmaxWarps;
 constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
 constexpr int kTcVWarp = kTcSoftmaxWarps + 2;
@@ -49,6 +52,9 @@ template <int D, bool Lite = false>
 struct TcSmem {
   static constexpr int kKStages = Lite ? 1 : (D == 128 ? 6 : 8);
   static constexpr int kVStages = Lite ? 1 : (D == 128 ? 5 : 8);
+  // S and P buffers in TMEM: three of each, so S(t + 2) can be computed while the softmax
+  // of tile t + 1 runs and the PV of tile t has not been issued yet
+  static constexpr int kSBufs = 3;
   static constexpr int kTile = kAttnKeys * D * 2;  // one K or V tile (D/64 boxes of 64 x 128 B)
   static constexpr int kQ = kTcRows * D * 2;        // D/64 boxes of 128 rows x 128 B
   static constexpr int kQOff = 0;
@@ -56,20 +62,20 @@ struct TcSmem {
   static constexpr int kVOff = kKOff + kKStages * kTile;
   static constexpr int kAncOff = kVOff + kVStages * kTile;
   static constexpr int kParOff = kAncOff + 64 * 8;
-  // row-maximum exchange [tile parity][half][row] and, after the loop, the denominator
-  // exchange [2][half][row]: three [2][128] float regions
+  // row-maximum exchange [tile parity][part][row] and, after the loop, the denominator
+  // exchange [part][row]
   static constexpr int kXchOff = kParOff + 64 * 4;
-  static constexpr int kBarOff = kXchOff + 3 * 2 * kTcRows * 4;
-  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], s_free[2],
-  // p_full[2], pv_done[2], o_final
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kBarOff = kXchOff + 3 * kTcParts * kTcRows * 4;
+  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[3], s_free[3],
+  // p_full[3], pv_done[3], o_final
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * kSBufs + 1;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  // TMEM columns: S0 [0, 64), S1 [64, 128), O [128, 128 + D), P0 / P1 32 columns each
+  // TMEM columns: S0-S2 64 columns each [0, 192), O [192, 192 + D), P0-P2 32 columns each
   // (64 bf16 per row, two to a column) after O
-  static constexpr uint32_t kOCol = 128;
-  static constexpr uint32_t kPCol = 128 + D;
-  static constexpr uint32_t kTmemCols = D == 128 ? 512 : 256;
+  static constexpr uint32_t kOCol = kSBufs * kAttnKeys;
+  static constexpr uint32_t kPCol = kOCol + D;
+  static constexpr uint32_t kTmemCols = 512;
 };
 
 struct TcAttnParams {
@@ -98,11 +104,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* k_empty = k_full + SK;
   uint64_t* v_full = k_empty + SK;
   uint64_t* v_empty = v_full + SV;
+  constexpr int NS = SM::kSBufs;
   uint64_t* s_full = v_empty + SV;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* o_final = pv_done + 2;
+  uint64_t* s_free = s_full + NS;
+  uint64_t* p_full = s_free + NS;
+  uint64_t* pv_done = p_full + NS;
+  uint64_t* o_final = pv_done + NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -141,7 +148,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
       mbar_init(smem_u32(&s_free[i]), 32 * kTcSoftmaxWarps);
       mbar_init(smem_u32(&p_full[i]), 32 * kTcSoftmaxWarps);
@@ -210,12 +217,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t o_tmem = tmem + SM::kOCol;
       bool ok = mbar_wait(smem_u32(q_full), 0, kErrAttnMmaWait);
       auto issue_s = [&](int t) {
-        const int s = t % SK;
+        const int s = t % SK, sb = t % NS;
         ok = ok && mbar_wait(smem_u32(&k_full[s]), (t / SK) & 1, kErrAttnMmaWait);
-        if (t >= 2) ok = ok && mbar_wait(smem_u32(&s_free[t & 1]), ((t - 2) >> 1) & 1, kErrAttnMmaWait);
+        if (t >= NS) ok = ok && mbar_wait(smem_u32(&s_free[sb]), (t / NS - 1) & 1, kErrAttnMmaWait);
         tc_fence_after();
         const uint32_t kb = k_stage(s);
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>((t & 1) * kAttnKeys);
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(sb * kAttnKeys);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int h = kk >> 2, k4 = kk & 3;
@@ -223,18 +230,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t bdesc = smem_desc_k_sw128(kb + h * kAttnKeys * 128) + 2 * k4;
           if (ok) tc_mma_f16(d_tmem, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[t & 1]));
+        tc_commit(smem_u32(&s_full[sb]));
         tc_commit(smem_u32(&k_empty[s]));  // the K slot is free once S(t) has read it
       };
+      // S runs two tiles ahead of PV: S(t + 2) is queued as soon as its buffer and K tile
+      // are free, before PV(t) waits for the softmax of tile t
       if (T > 0) issue_s(0);
+      if (T > 1) issue_s(1);
       for (int t = 0; t < T; ++t) {
-        if (t + 1 < T) issue_s(t + 1);
-        const int s = t % SV;
-        ok = ok && mbar_wait(smem_u32(&p_full[t & 1]), (t >> 1) & 1, kErrAttnMmaWait);
+        if (t + 2 < T) issue_s(t + 2);
+        const int s = t % SV, pb = t % NS;
+        ok = ok && mbar_wait(smem_u32(&p_full[pb]), (t / NS) & 1, kErrAttnMmaWait);
         ok = ok && mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnMmaWait);
         tc_fence_after();
         const uint32_t vb = v_stage(s);
-        const uint32_t pa = tmem + SM::kPCol + static_cast<uint32_t>((t & 1) * 32);
+        const uint32_t pa = tmem + SM::kPCol + static_cast<uint32_t>(pb * 32);
 #pragma unroll
         for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
           // 16 keys = 8 TMEM columns of P (bf16 pairs) and two 8-key groups of 1024 B of V;
@@ -242,7 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t bdesc = smem_desc_mn_sw128(vb + kk * 2048, kAttnKeys * 128, 1024);
           if (ok) tc_mma_f16_ts(o_tmem, pa + 8 * kk, bdesc, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(smem_u32(&pv_done[t & 1]));
+        tc_commit(smem_u32(&pv_done[pb]));
         tc_commit(smem_u32(&v_empty[s]));
       }
       tc_commit(smem_u32(o_final));
@@ -250,19 +260,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax warps
     constexpr int kSoftThreads = 32 * kTcSoftmaxWarps;
+    constexpr int C = kTcCols;              // score columns of this thread
+    constexpr int OC = D / kTcParts;        // output columns of this thread
     const int quarter = warp & 3;           // TMEM lane quarter = row block of 32
-    const int half = warp >> 2;             // which 32 of the 64 scores, which half of O
+    const int part = warp >> 2;             // which C of the 64 scores, which OC of O
     const int r = quarter * 32 + lane;      // query row = TMEM lane
     const int node = i0 + r / G;
     const int head = kvh * G + r % G;
     const bool rvalid = r < rows_blk && node < N;
     // a warp with no real row skips the score and output work (its rows of P and O are
-    // never read for an output), but keeps every barrier
+    // never read for an output), but keeps every barrier; the warps of a quarter cover the
+    // same rows, so they are live together
     const bool live = __any_sync(0xffffffffu, rvalid);
     const int tid = threadIdx.x;            // 0 .. kSoftThreads-1
     float* xch = reinterpret_cast<float*>(smem + SM::kXchOff);
-    const uint32_t pair_bar = 2 + quarter;  // named barrier of the two warps sharing a row
-    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
+    const uint32_t quarter_bar = 2 + quarter;  // named barrier of the warps sharing a quarter
+    auto quarter_sync = [&]() {
+      asm volatile("bar.sync %0, %1;" ::"r"(quarter_bar), "r"(32 * kTcParts) : "memory");
+    };
     if (last) {
       if (tid < N) {
         // ancestor bitmask: node tid and every node up its parent chain (a link that does
@@ -279,57 +294,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // named barrier of the softmax warps: the masks are read below
       asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
     }
-    // this thread's 32 key columns of the tree tile, as a bit mask
+    constexpr uint32_t kColMask = C == 32 ? 0xffffffffu : ((1u << C) - 1u);
+    // this thread's C key columns of the tree tile, as a bit mask
     const uint32_t tree_bits =
-        (last && rvalid) ? static_cast<uint32_t>(anc[node] >> (32 * half)) : 0u;
+        (last && rvalid) ? static_cast<uint32_t>(anc[node] >> (C * part)) & kColMask : 0u;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     float m_ref = -INFINITY, l = 0.f;
     for (int t = 0; t < T; ++t) {
       const bool tree = t >= nt;
-      mbar_wait(smem_u32(&s_full[t & 1]), (t >> 1) & 1, kErrAttnConsumerWait);
+      const int sb = t % NS;
+      mbar_wait(smem_u32(&s_full[sb]), (t / NS) & 1, kErrAttnConsumerWait);
       tc_fence_after();
-      uint32_t sv[32];
+      uint32_t sv[C];
       if (live) {
         __syncwarp();  // the TMEM load below is warp-wide
-        tmem_ld_32x32b_x32(lane_base + (t & 1) * kAttnKeys + 32 * half, sv);
+        tmem_ld_cols<C>(lane_base + sb * kAttnKeys + C * part, sv);
         tmem_ld_wait();
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[t & 1]));
+      mbar_arrive(smem_u32(&s_free[sb]));
       if (live) {
-        // visibility of this thread's 32 keys
-        uint32_t vis;
-        if (tree) {
-          vis = tree_bits & (N - 32 * half >= 32 ? 0xffffffffu
-                                                 : (N - 32 * half <= 0 ? 0u : ((1u << (N - 32 * half)) - 1u)));
-        } else {
-          const int valid = min(kAttnKeys, L - (t_begin + t) * kAttnKeys) - 32 * half;
-          vis = valid >= 32 ? 0xffffffffu : (valid <= 0 ? 0u : ((1u << valid) - 1u));
-        }
+        // visibility of this thread's C keys
+        const int first = tree ? 0 : (t_begin + t) * kAttnKeys;
+        const int valid = (tree ? N : min(kAttnKeys, L - first)) - C * part;
+        uint32_t vis = valid >= C ? kColMask : (valid <= 0 ? 0u : ((1u << valid) - 1u));
+        if (tree) vis &= tree_bits;
         if (!rvalid) vis = 0u;
         // raw scores; masked ones (past L_b, outside the ancestor set, padding rows) become
         // -inf, which also drops any non-finite value the padding holds
-        float x[32];
+        float x[C];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sv[j]);
-        if (vis != 0xffffffffu) {
+        for (int j = 0; j < C; ++j) x[j] = __uint_as_float(sv[j]);
+        if (vis != kColMask) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) x[j] = ((vis >> j) & 1u) ? x[j] : -INFINITY;
+          for (int j = 0; j < C; ++j) x[j] = ((vis >> j) & 1u) ? x[j] : -INFINITY;
         }
-        // tile maximum by a tree (short dependency chains: two warps share an SM
-        // sub-partition, so each warp's own instruction-level parallelism matters)
-        float mx[8];
+        // tile maximum by a tree (short dependency chains)
+        float mx[C / 4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) mx[j] = fmaxf(fmaxf(x[j], x[j + 8]), fmaxf(x[j + 16], x[j + 24]));
+        for (int j = 0; j < C / 4; ++j)
+          mx[j] = fmaxf(fmaxf(x[j], x[j + C / 4]), fmaxf(x[j + C / 2], x[j + 3 * C / 4]));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mx[j] = fmaxf(mx[j], mx[j + 4]);
-        float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        // row maximum of the tile: combine with the partner warp's half (the partner warp
-        // covers the same rows, so it is live exactly when this one is); in scaled log2
+        for (int w2 = C / 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+        float tmax = mx[0];
+        // row maximum of the tile: combine with the other parts of the row; in scaled log2
         // units (the scale is positive, so the maximum commutes with it)
-        xch[((t & 1) * 2 + half) * kTcRows + r] = tmax;
-        pair_sync();
-        tmax = fmaxf(tmax, xch[((t & 1) * 2 + (half ^ 1)) * kTcRows + r]) * prm.scale_log2;
+        xch[((t & 1) * kTcParts + part) * kTcRows + r] = tmax;
+        quarter_sync();
+#pragma unroll
+        for (int o = 1; o < kTcParts; ++o)
+          tmax = fmaxf(tmax, xch[((t & 1) * kTcParts + ((part + o) % kTcParts)) * kTcRows + r]);
+        tmax *= prm.scale_log2;
         const float m_new = fmaxf(m_ref, tmax);
         const bool rebase =
             m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kTcRescaleThreshold);
@@ -337,18 +354,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float f = scale_o ? fast_exp2(m_ref - m_new) : 1.0f;
         // TMEM loads/stores are warp-wide: the warp rescales if any of its rows must
         if (__any_sync(0xffffffffu, scale_o)) {
-          mbar_wait(smem_u32(&pv_done[(t - 1) & 1]), ((t - 1) >> 1) & 1, kErrAttnConsumerWait);
+          mbar_wait(smem_u32(&pv_done[(t - 1) % NS]), ((t - 1) / NS) & 1, kErrAttnConsumerWait);
           tc_fence_after();
           __syncwarp();
-#pragma unroll 1
-          for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
-            uint32_t ov[32];
-            tmem_ld_32x32b_x32(lane_base + SM::kOCol + c, ov);
-            tmem_ld_wait();
+          uint32_t ov[OC];
+          tmem_ld_cols<OC>(lane_base + SM::kOCol + OC * part, ov);
+          tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-            tmem_st_32x32b_x32(lane_base + SM::kOCol + c, ov);
-          }
+          for (int k = 0; k < OC; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+          tmem_st_cols<OC>(lane_base + SM::kOCol + OC * part, ov);
           tmem_st_wait();
         }
         if (rebase) {
@@ -359,12 +373,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // exp2(-inf) = 0 (and m = 0 while every key so far was masked)
         const float c = prm.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-        // P buffer t&1 was last read by PV(t - 2)
-        if (t >= 2) mbar_wait(smem_u32(&pv_done[t & 1]), ((t - 2) >> 1) & 1, kErrAttnConsumerWait);
-        uint32_t w[16];
+        // P buffer t % 3 was last read by PV(t - 3)
+        if (t >= NS) mbar_wait(smem_u32(&pv_done[sb]), (t / NS - 1) & 1, kErrAttnConsumerWait);
+        uint32_t w[C / 2];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < C / 2; ++e) {
           const float p0 = fast_exp2(fmaf(x[2 * e], c, neg_m));
           const float p1 = fast_exp2(fmaf(x[2 * e + 1], c, neg_m));
           w[e] = pack_bf16x2(p0, p1);
@@ -374,7 +388,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         __syncwarp();
-        tmem_st_32x32b_x16(lane_base + SM::kPCol + (t & 1) * 32 + 16 * half, w);
+        tmem_st_cols<C / 2>(lane_base + SM::kPCol + sb * 32 + (C / 2) * part, w);
         tmem_st_wait();
       }
       if (!tree) {
@@ -394,15 +408,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&p_full[t & 1]));
+      mbar_arrive(smem_u32(&p_full[sb]));
     }
 
     // ------------------------------------------------------------ epilogue
-    // row denominator: this thread's columns plus the partner's
+    // row denominator: this thread's columns plus the other parts'
     if (live) {
-      xch[(4 + half) * kTcRows + r] = l;
-      pair_sync();
-      l += xch[(4 + (half ^ 1)) * kTcRows + r];
+      float* lx = xch + 2 * kTcParts * kTcRows;
+      lx[part * kTcRows + r] = l;
+      quarter_sync();
+#pragma unroll
+      for (int o = 1; o < kTcParts; ++o) l += lx[((part + o) % kTcParts) * kTcRows + r];
     }
     if (T > 0) {
       mbar_wait(smem_u32(o_final), 0, kErrAttnConsumerWait);
@@ -412,38 +428,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool single = prm.num_splits == 1;
     const float inv = (l > 0.f) ? 1.0f / l : 0.f;
     if (live) {
-      for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
-        uint32_t ov[32];
-        __syncwarp();  // the TMEM load below is warp-wide
-        if (T > 0) {
-          tmem_ld_32x32b_x32(lane_base + SM::kOCol + c, ov);
-          tmem_ld_wait();
-        } else {
+      uint32_t ov[OC];
+      __syncwarp();  // the TMEM load below is warp-wide
+      if (T > 0) {
+        tmem_ld_cols<OC>(lane_base + SM::kOCol + OC * part, ov);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) ov[k] = 0u;
+        for (int k = 0; k < OC; ++k) ov[k] = 0u;
+      }
+      const int c0 = OC * part;
+      if (!rvalid) {
+      } else if (single) {
+        uint4* dst = reinterpret_cast<uint4*>(prm.out + prow_g * D + c0);
+#pragma unroll
+        for (int k = 0; k < OC; k += 8) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(ov[k + 2]) * inv, __uint_as_float(ov[k + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(ov[k + 4]) * inv, __uint_as_float(ov[k + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(ov[k + 6]) * inv, __uint_as_float(ov[k + 7]) * inv);
+          dst[k / 8] = w;
         }
-        if (!rvalid) {
-        } else if (single) {
-          uint4* dst = reinterpret_cast<uint4*>(prm.out + prow_g * D + c);
+      } else {
+        float4* dst = reinterpret_cast<float4*>(prm.part_acc + (prow_g * prm.num_splits + split) * D + c0);
 #pragma unroll
-          for (int k = 0; k < 32; k += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ov[k + 2]) * inv, __uint_as_float(ov[k + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ov[k + 4]) * inv, __uint_as_float(ov[k + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ov[k + 6]) * inv, __uint_as_float(ov[k + 7]) * inv);
-            dst[k / 8] = w;
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(prm.part_acc + (prow_g * prm.num_splits + split) * D + c);
-#pragma unroll
-          for (int k = 0; k < 32; k += 4)
-            dst[k / 4] = make_float4(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1]),
-                                     __uint_as_float(ov[k + 2]), __uint_as_float(ov[k + 3]));
-        }
+        for (int k = 0; k < OC; k += 4)
+          dst[k / 4] = make_float4(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1]),
+                                   __uint_as_float(ov[k + 2]), __uint_as_float(ov[k + 3]));
       }
     }
-    if (rvalid && !single && half == 0)
+    if (rvalid && !single && part == 0)
       *reinterpret_cast<float2*>(prm.part_ml + (prow_g * prm.num_splits + split) * 2) = make_float2(m_ref, l);
   }
 

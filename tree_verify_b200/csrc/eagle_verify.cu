@@ -282,8 +282,6 @@ bool ensure_attributes(int dev) {
                                227 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(lm_head_tc_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(lm_head_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               227 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TcSmem<64>::kAlloc) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -450,65 +448,13 @@ eagle_status_t run_lm_head_persistent(const eagle_shape_t* s, const void* hidden
   if (!encode_bf16(&tw, w, 2, wd, stride, wbox) || !encode_bf16(&th, hidden, 2, hd, stride, hbox))
     return EAGLE_ERR_CUDA;
   const int vtiles = (V + kLmBlockV - 1) / kLmBlockV;
-  // hidden boxes mostly hit L2: a short ring; W boxes come from HBM: the rest of the
-  // shared memory, so they are issued several k-blocks ahead
-  const int hstages = kLmpHiddenStages;
-  int wstages = 2;
-  while (wstages < kLmpMaxStages && lmp_smem_bytes(plan.bn, wstages + 1, hstages) <= 220 * 1024) ++wstages;
-  LmpParams prm{logits, M, V, H, plan.bn, plan.chunks, vtiles, wstages, hstages};
-  const size_t smem = lmp_smem_bytes(plan.bn, wstages, hstages);
+  int stages = 2;
+  while (stages < 8 && lmp_smem_bytes(plan.bn, stages + 1) <= 220 * 1024) ++stages;
+  LmpParams prm{logits, M, V, H, plan.bn, plan.chunks, vtiles, stages};
+  const size_t smem = lmp_smem_bytes(plan.bn, stages);
   const long tiles = static_cast<long>(vtiles) * plan.chunks;
   const int grid = static_cast<int>(tiles < kNumSMs ? tiles : kNumSMs);
   lm_head_tc_persist_kernel<<<grid, kLmpThreads, smem, st>>>(tw, th, prm);
-  return launch_status();
-}
-
-// The CTA-pair kernel: tree rows in chunks of a multiple of 32 (each CTA of a pair holds
-// half of a chunk), picked to waste the fewest padded rows.
-eagle_status_t run_lm_head_pair(const eagle_shape_t* s, const void* hidden, const void* w,
-                                float* logits, cudaStream_t st) {
-  const int M = s->batch * s->num_nodes, V = s->vocab, H = s->hidden;
-  int chunks = (M + 255) / 256, bn = 0;
-  long best = -1;
-  for (int c = chunks; c <= chunks + 2; ++c) {
-    const int b = ((M + c - 1) / c + 31) / 32 * 32;
-    if (b > 256) continue;
-    if (best < 0 || static_cast<long>(c) * b < best) {
-      best = static_cast<long>(c) * b;
-      chunks = c;
-      bn = b;
-    }
-  }
-  CUtensorMap tw, th;
-  const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
-  const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};
-  const cuuint64_t stride[1] = {static_cast<cuuint64_t>(H) * 2};
-  const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(kLmBlockV)};
-  const cuuint32_t hbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(bn / 2)};
-  if (!encode_bf16(&tw, w, 2, wd, stride, wbox) || !encode_bf16(&th, hidden, 2, hd, stride, hbox))
-    return EAGLE_ERR_CUDA;
-  const int vpairs = (V + 2 * kLmBlockV - 1) / (2 * kLmBlockV);
-  int stages = 2;
-  while (stages < 12 && lm2_smem_bytes(bn, stages + 1) <= 220 * 1024) ++stages;
-  Lm2Params prm{logits, M, V, H, bn, chunks, vpairs, stages};
-  const long tiles = static_cast<long>(vpairs) * chunks;
-  const int pairs = static_cast<int>(tiles < kNumSMs / 2 ? tiles : kNumSMs / 2);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(kLm2Threads);
-  cfg.dynamicSmemBytes = lm2_smem_bytes(bn, stages);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, lm_head_tc_pair_kernel, tw, th, prm) != cudaSuccess) {
-    cudaGetLastError();
-    return EAGLE_ERR_CUDA;
-  }
   return launch_status();
 }
 
@@ -524,11 +470,7 @@ eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const voi
     return launch_status();
   }
   const LmPlan plan = plan_lm_head(s, max_stages);
-#ifdef EAGLE_LM_PAIR
-  if (plan.chunks > 1 && started == nullptr) return run_lm_head_pair(s, hidden, w, logits, st);
-#else
   if (plan.chunks > 1 && started == nullptr) return run_lm_head_persistent(s, hidden, w, logits, st, plan);
-#endif
   CUtensorMap tw, th;
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
   const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};

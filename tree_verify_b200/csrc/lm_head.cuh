@@ -172,20 +172,13 @@ __global__ void __launch_bounds__(kLmThreads, 1)
 // the weight stream): one CTA per SM walks a list of (vocabulary tile, row chunk) tiles,
 // row chunk fastest, so the CTAs working on the chunks of one vocabulary tile run side by
 // side and W is read from HBM about once.  Two TMEM accumulators (2 x 256 columns) let the
-// epilogue warps drain tile j while the MMAs of tile j + 1 run.  W boxes (from HBM) and
-// hidden boxes (L2-resident) fill rings of their own, the W ring deeper, so the slower
-// stream is issued further ahead.  Warp roles: warp 0 lane 0 issues the W loads, warp 2
-// lane 0 the hidden loads, warp 1 owns TMEM and lane 0 issues the MMAs, warps 3-6 drain
-// TMEM (warp w reads TMEM lanes 32 * (w % 4) ..) and store fp32 logits in coalesced
-// 128-byte rows.
+// epilogue warps drain tile j while the MMAs of tile j + 1 run.  Warp roles: warp 0 lane 0
+// issues TMA (a W box and a hidden box per k block, one ring), warp 1 owns TMEM and lane 0
+// issues the MMAs, warps 2-5 drain TMEM (warp w reads TMEM lanes 32 * (w % 4) ..) and store
+// fp32 logits in coalesced 128-byte rows.
 
-constexpr int kLmpThreads = 224;
+constexpr int kLmpThreads = 192;
 constexpr int kLmpAccCols = 256;  // columns per accumulator
-constexpr int kLmpMaxStages = 12;
-#ifndef EAGLE_LMP_HIDDEN_STAGES
-#define EAGLE_LMP_HIDDEN_STAGES 3
-#endif
-constexpr int kLmpHiddenStages = EAGLE_LMP_HIDDEN_STAGES;  // hidden ring depth (tuning constant)
 
 struct LmpParams {
   float* logits;
@@ -193,13 +186,11 @@ struct LmpParams {
   int32_t bn;       // rows per chunk, multiple of 16, <= 256
   int32_t chunks;   // row chunks (ceil(M / bn))
   int32_t vtiles;   // vocabulary tiles of 128
-  int32_t wstages;  // W ring depth (16 KB slots)
-  int32_t hstages;  // hidden ring depth (bn * 128 B slots)
+  int32_t stages;
 };
 
-__host__ __device__ inline size_t lmp_smem_bytes(int bn, int wstages, int hstages) {
-  return 1024 + static_cast<size_t>(wstages) * kLmBlockV * kLmBlockK * 2 +
-         static_cast<size_t>(hstages) * bn * kLmBlockK * 2 + (2 * wstages + 2 * hstages + 5) * 8 + 16;
+__host__ __device__ inline size_t lmp_smem_bytes(int bn, int stages) {
+  return 1024 + static_cast<size_t>(stages) * lm_stage_bytes(bn) + (2 * stages + 5) * 8 + 16;
 }
 
 __global__ void __launch_bounds__(kLmpThreads, 1)
@@ -208,18 +199,14 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
   extern __shared__ uint8_t lmp_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lmp_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int SW = prm.wstages, SH = prm.hstages;
+  const int S = prm.stages;
   const int bn = prm.bn;
-  constexpr uint32_t kWBytes = kLmBlockV * kLmBlockK * 2;
-  const uint32_t h_bytes = static_cast<uint32_t>(bn) * kLmBlockK * 2;
-  uint8_t* a_tiles = smem;                       // SW x 16 KB
-  uint8_t* b_tiles = smem + SW * kWBytes;        // SH x bn*128 B
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_tiles + SH * h_bytes);
-  uint64_t* w_full = bars;
-  uint64_t* w_empty = w_full + SW;
-  uint64_t* h_full = w_empty + SW;
-  uint64_t* h_empty = h_full + SH;
-  uint64_t* acc_full = h_empty + SH;
+  uint8_t* a_tiles = smem;                                    // S x 16 KB
+  uint8_t* b_tiles = smem + S * kLmBlockV * kLmBlockK * 2;    // S x bn*128 B
+  uint64_t* bars = reinterpret_cast<uint64_t*>(b_tiles + S * bn * kLmBlockK * 2);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* acc_full = bars + 2 * S;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -233,13 +220,9 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_h);
-    for (int s = 0; s < SW; ++s) {
-      mbar_init(smem_u32(&w_full[s]), 1);
-      mbar_init(smem_u32(&w_empty[s]), 1);
-    }
-    for (int s = 0; s < SH; ++s) {
-      mbar_init(smem_u32(&h_full[s]), 1);
-      mbar_init(smem_u32(&h_empty[s]), 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&acc_full[a]), 1);
@@ -259,14 +242,10 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
   const uint32_t tmem = *tmem_slot;
   pdl_launch_dependents();
 
-  if (warp == 0 || warp == 2) {
+  if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producers: warp 0 the W boxes, warp 2 the hidden boxes
-      const bool is_w = warp == 0;
-      const int S = is_w ? SW : SH;
-      uint64_t* full = is_w ? w_full : h_full;
-      uint64_t* empty = is_w ? w_empty : h_empty;
-      const uint32_t bytes = is_w ? kWBytes : h_bytes;
+      // ---------------- TMA producer
+      const uint32_t bytes = lm_stage_bytes(bn);
       const uint64_t pol_h = l2_policy_evict_last();  // every tile re-reads hidden
       int it = 0, issued = 0;
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
@@ -279,10 +258,9 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
           }
           const uint32_t fb = smem_u32(&full[s]);
           mbar_arrive_expect_tx(fb, bytes);
-          if (is_w)
-            tma_load_2d(smem_u32(a_tiles + s * kWBytes), &tm_w, fb, kb * kLmBlockK, v0);
-          else
-            tma_load_2d_hint(smem_u32(b_tiles + s * h_bytes), &tm_h, fb, kb * kLmBlockK, c * bn, pol_h);
+          tma_load_2d(smem_u32(a_tiles + s * kLmBlockV * kLmBlockK * 2), &tm_w, fb, kb * kLmBlockK, v0);
+          tma_load_2d_hint(smem_u32(b_tiles + s * bn * kLmBlockK * 2), &tm_h, fb, kb * kLmBlockK, c * bn,
+                           pol_h);
           issued = it + 1;
         }
       }
@@ -305,20 +283,18 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(a * kLmpAccCols);
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int sw = it % SW, sh = it % SH;
-          if (!mbar_wait(smem_u32(&w_full[sw]), (it / SW) & 1, kErrLmMmaWait) ||
-              !mbar_wait(smem_u32(&h_full[sh]), (it / SH) & 1, kErrLmMmaWait)) {
+          const int s = it % S;
+          if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, kErrLmMmaWait)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t a_desc = smem_desc_k_sw128(smem_u32(a_tiles + sw * kWBytes));
-          const uint64_t b_desc = smem_desc_k_sw128(smem_u32(b_tiles + sh * h_bytes));
+          const uint64_t a_desc = smem_desc_k_sw128(smem_u32(a_tiles + s * kLmBlockV * kLmBlockK * 2));
+          const uint64_t b_desc = smem_desc_k_sw128(smem_u32(b_tiles + s * bn * kLmBlockK * 2));
 #pragma unroll
           for (int k = 0; k < kLmBlockK / 16; ++k)
             tc_mma_f16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-          tc_commit(smem_u32(&w_empty[sw]));
-          tc_commit(smem_u32(&h_empty[sh]));
+          tc_commit(smem_u32(&empty[s]));
         }
         if (!ok) {
           *abort_flag = 1;
@@ -330,7 +306,7 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
       tc_commit(smem_u32(mma_done));
     }
   } else {
-    // ---------------- epilogue: TMEM -> registers -> global (warps 3-6)
+    // ---------------- epilogue: TMEM -> registers -> global (warps 2-5)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int j = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++j) {
@@ -375,228 +351,11 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
   }
 }
 
-// ------------------------------------------------------------------ CTA-pair bf16 path
-// The tensor-bound shapes (more than 256 tree rows) on CTA pairs: a 2-CTA cluster computes
-// a 256-entry vocabulary tile x a chunk of bn tree rows with one pair-wide MMA per k step
-// (M = 256: each CTA supplies 128 W rows and half of the bn hidden rows, and receives its
-// 128 x bn accumulator in its own TMEM).  Per k block each CTA loads 16 KB of W and
-// bn/2 x 128 B of hidden -- two thirds of what a single CTA needs for the same work -- so
-// a ring of about six stages fits and the loads run well ahead of the MMAs.  Persistent:
-// a pair walks (vocabulary pair-tile, row chunk) tiles, chunk fastest, so the pairs working
-// on one vocabulary tile run side by side and W comes from HBM about once; two TMEM
-// accumulators let the epilogue of tile j run under the MMAs of tile j + 1.
-//   warp 0 lane 0   TMA for this CTA's halves; the completion of both CTAs' loads is
-//                   counted on the even CTA's `full` barrier (which the even CTA arms for
-//                   both);
-//   warp 1          TMEM (pair allocation); in the even CTA lane 0 issues the MMAs and
-//                   signals both CTAs' barriers with per-CTA commits;
-//   warps 2-5       epilogue from this CTA's TMEM; one arrival per warp on the even CTA's
-//                   `acc_empty`.
-// The CTAs leave together: each tells the other it is done, and waits (bounded) to hear it.
-
-constexpr int kLm2Threads = 192;
-constexpr int kLm2AccCols = 256;
-
-struct Lm2Params {
-  float* logits;
-  int32_t M, V, H;
-  int32_t bn;      // rows per chunk, multiple of 32, <= 256 (MMA N; each CTA holds bn / 2)
-  int32_t chunks;  // row chunks
-  int32_t vpairs;  // vocabulary tiles of 256
-  int32_t stages;
-};
-
-__host__ __device__ inline uint32_t lm2_stage_bytes(int bn) {
-  return static_cast<uint32_t>(kLmBlockV * kLmBlockK * 2 + (bn / 2) * kLmBlockK * 2);
-}
-__host__ __device__ inline size_t lm2_smem_bytes(int bn, int stages) {
-  return 1024 + static_cast<size_t>(stages) * lm2_stage_bytes(bn) + (2 * stages + 7) * 8 + 16;
-}
-
-__global__ void __launch_bounds__(kLm2Threads, 1)
-    lm_head_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
-                           const __grid_constant__ CUtensorMap tm_h, const Lm2Params prm) {
-  extern __shared__ uint8_t lm2_smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lm2_smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const int S = prm.stages;
-  const int bn = prm.bn, hb = prm.bn / 2;
-  constexpr uint32_t kWBytes = kLmBlockV * kLmBlockK * 2;
-  const uint32_t h_bytes = static_cast<uint32_t>(hb) * kLmBlockK * 2;
-  uint8_t* a_tiles = smem;                     // S x 16 KB
-  uint8_t* b_tiles = smem + S * kWBytes;       // S x hb*128 B
-  uint64_t* bars = reinterpret_cast<uint64_t*>(b_tiles + S * h_bytes);
-  uint64_t* full = bars;                       // even CTA: both CTAs' bytes of stage s
-  uint64_t* empty = bars + S;                  // stage s free again (each CTA its own)
-  uint64_t* acc_full = bars + 2 * S;           // accumulator a ready (each CTA its own)
-  uint64_t* acc_empty = acc_full + 2;          // even CTA: accumulator a drained by both
-  uint64_t* mma_done = acc_empty + 2;          // every MMA has completed (each CTA its own)
-  uint64_t* done = mma_done + 1;               // the other CTA is leaving
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const uint32_t peer = rank ^ 1u;
-  const bool even = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int KB = (prm.H + kLmBlockK - 1) / kLmBlockK;
-  const int num_tiles = prm.vpairs * prm.chunks;
-
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_w);
-    prefetch_tmap(&tm_h);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(smem_u32(&acc_full[a]), 1);
-      mbar_init(smem_u32(&acc_empty[a]), 8);  // 4 epilogue warps x 2 CTAs
-    }
-    mbar_init(smem_u32(mma_done), 1);
-    mbar_init(smem_u32(done), 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), 2 * kLm2AccCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  // both CTAs' barriers are initialised before either signals the other's
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  pdl_launch_dependents();
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer (this CTA's W rows and half of the hidden rows)
-      const uint32_t bytes = kWBytes + h_bytes;
-      const uint32_t full_even = dsmem_map(smem_u32(&full[0]), 0);
-      const uint64_t pol_h = l2_policy_evict_last();  // every tile re-reads hidden
-      int it = 0;
-      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += npairs) {
-        const int c = tile % prm.chunks;
-        const int v0 = (tile / prm.chunks) * (2 * kLmBlockV) + static_cast<int>(rank) * kLmBlockV;
-        const int h0 = c * bn + static_cast<int>(rank) * hb;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % S, n = it / S;
-          if (n > 0 && !mbar_wait(smem_u32(&empty[s]), (n - 1) & 1, kErrLmProducerWait)) {
-            *abort_flag = 1;
-            break;
-          }
-          if (even) mbar_arrive_expect_tx(smem_u32(&full[s]), 2 * bytes);
-          const uint32_t fb = full_even + static_cast<uint32_t>(s) * 8u;
-          tma_load_2d_pair(smem_u32(a_tiles + s * kWBytes), &tm_w, fb, kb * kLmBlockK, v0);
-          tma_load_2d_pair_hint(smem_u32(b_tiles + s * h_bytes), &tm_h, fb, kb * kLmBlockK, h0, pol_h);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && even) {
-      // ---------------- MMA issuer (even CTA)
-      const uint32_t idesc = idesc_bf16_f32(2 * kLmBlockV, bn);
-      const uint32_t empty_own = smem_u32(&empty[0]), empty_peer = dsmem_map(empty_own, peer);
-      const uint32_t accf_own = smem_u32(&acc_full[0]), accf_peer = dsmem_map(accf_own, peer);
-      const uint32_t done_own = smem_u32(mma_done), done_peer = dsmem_map(done_own, peer);
-      int it = 0, j = 0;
-      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += npairs, ++j) {
-        const int a = j & 1;
-        if (j >= 2 && !mbar_wait(smem_u32(&acc_empty[a]), ((j - 2) >> 1) & 1, kErrLmMmaWait)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(a * kLm2AccCols);
-        bool ok = true;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(smem_u32(&full[s]), (it / S) & 1, kErrLmMmaWait)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t a_desc = smem_desc_k_sw128(smem_u32(a_tiles + s * kWBytes));
-          const uint64_t b_desc = smem_desc_k_sw128(smem_u32(b_tiles + s * h_bytes));
-#pragma unroll
-          for (int k = 0; k < kLmBlockK / 16; ++k)
-            tc_mma_f16_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-          tc_commit_pair(empty_own + static_cast<uint32_t>(s) * 8u);
-          tc_commit_pair(empty_peer + static_cast<uint32_t>(s) * 8u);
-        }
-        if (!ok) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_commit_pair(accf_own + static_cast<uint32_t>(a) * 8u);
-        tc_commit_pair(accf_peer + static_cast<uint32_t>(a) * 8u);
-      }
-      // orders both CTAs' TMEM release after every MMA issued
-      tc_commit_pair(done_own);
-      tc_commit_pair(done_peer);
-    }
-  } else {
-    // ---------------- epilogue: this CTA's TMEM -> registers -> global (warps 2-5)
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const uint32_t acce_even = dsmem_map(smem_u32(&acc_empty[0]), 0);
-    int j = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++j) {
-      const int a = j & 1;
-      if (!mbar_wait(smem_u32(&acc_full[a]), (j >> 1) & 1, kErrLmEpilogueWait)) {
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const int c = tile % prm.chunks;
-      const int v = (tile / prm.chunks) * (2 * kLmBlockV) + static_cast<int>(rank) * kLmBlockV + q * 32 + lane;
-      const int r0 = c * bn;
-      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * kLm2AccCols);
-      float* out = prm.logits;
-      for (int c0 = 0; c0 < bn; c0 += 16) {
-        uint32_t r[16];
-        __syncwarp();  // the TMEM load below is warp-wide
-        tmem_ld_32x32b_x16(lane_base + c0, r);
-        tmem_ld_wait();
-        if (v < prm.V) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int row = r0 + c0 + e;
-            if (row < prm.M) out[static_cast<size_t>(row) * prm.V + v] = __uint_as_float(r[e]);
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(acce_even + static_cast<uint32_t>(a) * 8u);
-    }
-  }
-  __syncwarp();
-  // every MMA (issued by the even CTA) has completed before TMEM is released
-  if (warp == 1 && lane == 0) mbar_wait(smem_u32(mma_done), 0, kErrLmMmaWait);
-  tc_fence_before();
-  __syncthreads();
-  // leave together: neither CTA's shared memory goes away while the other may still read it
-  // (the even CTA's MMAs read the odd CTA's tiles) or signal its barriers
-  if (threadIdx.x == 0) {
-    mbar_arrive_remote(dsmem_map(smem_u32(done), peer));
-    mbar_wait_cluster(smem_u32(done), 0, kErrLmEpilogueWait, 2 * kWaitLimitNs);
-  }
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem, 2 * kLm2AccCols);
-  }
-}
-
 // ------------------------------------------------------------------ fp32 SIMT path
 
 constexpr int kLmF32TileV = 64;
 constexpr int kLmF32TileR = 16;
-constexpr int kLmF32TileK = 32;
+constexpr int kLmF32TileK = 128;  // 41 KB of tiles: few dependent memory round trips per row
 
 __global__ void __launch_bounds__(256)
     lm_head_f32_kernel(const float* __restrict__ hidden, const float* __restrict__ w,

@@ -78,8 +78,8 @@ typedef struct {
 const char *eagle_status_string(eagle_status_t status);
 
 /* Bytes of `workspace` the entry points below need for this shape (0 if the shape is
- * invalid).  The split-KV partials of tree attention live there; for shapes that
- * eagle_verify_step may run beside the LM head this is the larger of the two split plans. */
+ * invalid, or if tree attention runs in a single split).  The split-KV partials of tree
+ * attention live there. */
 size_t eagle_workspace_bytes(const eagle_shape_t *shape);
 
 /*
@@ -169,12 +169,10 @@ eagle_status_t eagle_tree_accept(const eagle_shape_t *shape, const float *logits
  *
  * bf16: tree attention (whose output the walk does not read) and its split merge run on a
  * second stream of the library's own (one per device, created with two events on the first
- * bf16 call), and `stream` waits for them before any work enqueued after this call.  The
- * attention starts when the LM head completes and runs while the walk runs; greedy steps
- * (temperature 0) on shapes with few tree rows (B*N <= 48 at D = 128) start it beside the
- * LM head instead, once every LM-head CTA holds its SM.  bf16 calls on one device are
+ * bf16 call), starting when the LM head completes and running beside the walk; `stream`
+ * waits for them before any work enqueued after this call.  bf16 calls on one device are
  * serialised on the host while they are enqueued.  fp32: everything on `stream`, tree
- * attention after the walk.  The workspace from eagle_workspace_bytes() covers both plans.
+ * attention after the walk.
  */
 eagle_status_t eagle_verify_step(const eagle_shape_t *shape, const void *q,
                                  const void *k_prefix, const void *v_prefix,

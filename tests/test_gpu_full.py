@@ -66,11 +66,7 @@ def test_verify_step_full_size(cuda_lib, orc, name, T):
     assert st.compared >= 0.75 * st.decisions, st
 
 
-def _align256(x):
-    return (x + 255) // 256 * 256
-
-
-OVERLAP_CASES = {
+STEP_CASES = {
     # one sequence, the bench workload's tree (45 nodes) on a shorter prefix
     "vicuna": ("vicuna7b_static", dict(prefix_len=700, vocab=5000, hidden=1024)),
     # two sequences of ragged length, a random tree of 20 nodes
@@ -82,29 +78,23 @@ OVERLAP_CASES = {
 }
 
 
-@pytest.mark.parametrize("case", sorted(OVERLAP_CASES))
-def test_verify_step_overlapped_schedule(cuda_lib, orc, case):
-    """Shapes small enough for eagle_verify_step's two-stream schedule (greedy steps:
-    attention in one-tile-per-CTA splits beside the LM head): logits and the walk are
-    bit-identical to the stage calls; the attention, merged from other splits, matches the
-    oracle and the standalone call within the bf16 tolerance."""
-    from tree_verify_b200 import binding
+@pytest.mark.parametrize("case", sorted(STEP_CASES))
+@pytest.mark.parametrize("T", [0.0, 1.0])
+def test_verify_step_two_stream_schedule(cuda_lib, orc, case, T):
+    """eagle_verify_step's two-stream schedule (attention and its merge on the library's
+    side stream, beside the walk) gives the same logits and walk bits as the stage calls in
+    sequence, and attention that matches the oracle and the stand-alone call."""
     from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
-    base, kw = OVERLAP_CASES[case]
+    base, kw = STEP_CASES[case]
     w = wl.scaled(wl.WORKLOADS[base], **kw)
-    inp = wl.generate(w, 1.0)
+    inp = wl.generate(w, T)
     shape = shape_from_workload(w)
-    # the workspace is sized for the one-tile-per-CTA plan: the schedule is the overlapped one
-    rows = w.batch * w.num_nodes * w.num_q_heads
-    splits = (w.prefix_len + 63) // 64 + 1
-    assert binding.workspace_bytes(shape) == (_align256(rows * splits * w.head_dim * 4)
-                                              + _align256(rows * splits * 2 * 4))
     x = StepInputs.from_numpy(inp, w.dtype)
     a, b = VerifyStep(shape), VerifyStep(shape)
-    a.run(x, 0.0, 3, 4)  # the schedule that overlaps attention with the LM head is greedy-only
+    a.run(x, T, 3, 4)
     b.attention(x)
     b.lm_head(x)
-    b.accept(x, 0.0, 3, 4)
+    b.accept(x, T, 3, 4)
     torch.cuda.synchronize()
     assert cuda_lib.device_error(reset=True) == 0
     for name in ("logits", "accepted_nodes", "accept_len", "next_token"):
@@ -120,7 +110,7 @@ def test_verify_step_overlapped_schedule(cuda_lib, orc, case):
 
 def test_verify_step_stages_equal_fused_call(cuda_lib):
     """The three stage entry points in sequence give the same bits as eagle_verify_step
-    (a shape with too many tree rows for the overlapped schedule)."""
+    (three sequences of ragged length)."""
     from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
     w = wl.scaled(wl.WORKLOADS["batched7b"], batch=3, prefix_len=700, prefix_min=100, vocab=5000,
                   hidden=1024)

@@ -375,13 +375,16 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
   const float invT = T > 0.f ? 1.0f / T : 0.f;
   // does this CTA own vocabulary entry x (and is x a real token)?
   auto owns = [&](int x) { return x >= v_lo && x < v_lo + n_loc; };
-  auto fetch_q = [&](int qb, int c) {
-    fetch_slice<kBulk>(qbuf + qb * slice, prm.draft + (seq + c) * V + v_lo, n_loc, &sh.q_bar[qb]);
-    if (kBulk && n_loc > 0) pending |= 1u << qb;
-  };
   auto wait_q = [&](int qb) {
     if (!kBulk || (pending >> qb) & 1u) failed |= !wait_slice<kBulk>(&sh.q_bar[qb], q_phase[qb], n_loc);
     pending &= ~(1u << qb);
+  };
+  // a buffer whose previous copy is still in flight (a prefetch for a candidate that was
+  // never tested) is landed before it is refilled
+  auto fetch_q = [&](int qb, int c) {
+    if (kBulk && ((pending >> qb) & 1u)) wait_q(qb);
+    fetch_slice<kBulk>(qbuf + qb * slice, prm.draft + (seq + c) * V + v_lo, n_loc, &sh.q_bar[qb]);
+    if (kBulk && n_loc > 0) pending |= 1u << qb;
   };
   // this CTA will push nothing more: tell every peer (lane l of warp 0 made every push to
   // peer l, so its arrival also releases them)
@@ -396,6 +399,13 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     const int c_begin = sh.child_start[node];
     const int kids = sh.child_start[node + 1] - c_begin;
     const int pre = min(kids, NQ);
+    // buffers still holding an untested candidate's copy: every thread sees it land before
+    // one thread re-arms the barrier (a thread polling after the next phase completed would
+    // otherwise wait for a phase that never comes)
+    if (kBulk && (pending & ((1u << pre) - 1u))) {
+      for (int j = 0; j < pre; ++j) wait_q(j);
+      __syncthreads();
+    }
     for (int j = 0; j < pre; ++j) fetch_q(j, sh.child_list[c_begin + j]);
     if (tid < kids) {
       const int c = sh.child_list[c_begin + tid];
@@ -574,10 +584,9 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       const int c = sh.child_list[c_begin + j_acc];
       if (tid == 0) sh.acc_nodes[nacc] = c;
       ++nacc;
-      // candidates [j_acc, j_acc + NQ) may still have draft-row copies in flight: land them
-      // before their buffers are reused
-      if (kBulk)
-        for (int j = j_acc; j < min(kids, j_acc + NQ); ++j) wait_q(j % NQ);
+      // candidates [j_acc, j_acc + NQ) may still have draft-row copies in flight: they stay
+      // pending until their buffers are refilled (or the walk ends), so the next node's
+      // row request does not wait for them
       __syncthreads();
       cur = c;
       continue;

@@ -8,7 +8,7 @@
 // i to the root (i included).
 //
 // This file holds what both precisions share (parameters, the 128-byte-swizzled tile
-// layout of 64-key K/V tiles), the log-sum-exp merge of split partials, and the fp32
+// layout of 128-key K/V tiles), the log-sum-exp merge of split partials, and the fp32
 // path.  The bf16 path runs on the tensor cores (attention_tc.cuh).
 //
 // f32 path: one warp per output row, fp32 SIMT, keys streamed in order (small shapes).
@@ -18,7 +18,7 @@
 
 namespace eagle {
 
-constexpr int kAttnKeys = 64;        // keys per tile
+constexpr int kAttnKeys = 128;       // keys per tile
 
 struct AttnParams {
   const __nv_bfloat16* q;       // [B,N,Hq,D]
@@ -34,8 +34,8 @@ struct AttnParams {
   float scale_log2;             // softmax scale * log2(e)
 };
 
-// Byte offset of element (row, d) in a 64-row tile stored as D/64 boxes of [64][64] bf16
-// with the 128-byte swizzle (16-byte chunk index XOR row % 8).
+// Byte offset of element (row, d) in a kAttnKeys-row tile stored as D/64 boxes of
+// [kAttnKeys][64] bf16 with the 128-byte swizzle (16-byte chunk index XOR row % 8).
 __device__ __forceinline__ uint32_t attn_swz(int row, int d) {
   const int half = d >> 6;
   const int chunk = (d & 63) >> 3;

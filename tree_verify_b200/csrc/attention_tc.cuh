@@ -7,27 +7,29 @@
 // r -> node i0 + r / G, head kvh*G + r % G), so one 128-row MMA tile covers all of them and
 // every prefix K/V tile is read from HBM once.
 //
-//   warp 16 (lane 0)  TMA: the Q tile once (a 3-D box over [B*N, Hq, D]) and the 64-key K
+//   warp 16 lane 0    TMA: the Q tile once (a 3-D box over [B*N, Hq, D]) and the 128-key K
 //                     tiles of this split into the K ring;
-//   warp 18 (lane 0)  TMA: the matching V tiles into the V ring (its own ring and barriers,
+//   warp 16 lane 1    TMA: the matching V tiles into the V ring (its own ring and barriers,
 //                     so a K slot is refilled as soon as S = Q K^T has read it, a tile
 //                     earlier than its V slot);
-//   warp 17 (lane 0)  tcgen05.mma: S = Q K^T (M 128, N 64, K = D) into one of two TMEM
-//                     buffers, then O += P V (M 128, N = D, K 64) with P read from TMEM and
-//                     V as an MN-major operand straight from its TMA tile;
+//   warp 17 (lane 0)  tcgen05.mma: S = Q K^T (M 128, N 128, K = D) into one of two TMEM
+//                     buffers, then O += P V (M 128, N = D, K 128) with P read from TMEM and
+//                     V as an MN-major operand straight from its TMA tile (128-key tiles:
+//                     fewer, larger MMA instructions per key);
 //   warps 0-15        four threads per query row (= TMEM lane): warps w, w + 4, w + 8 and
-//                     w + 12 share the lane quarter w % 4 and take 16 of the tile's 64 scores
+//                     w + 12 share the lane quarter w % 4 and take 32 of the tile's 128 scores
 //                     each (tcgen05.ld), mask them (prefix length, or the ancestor bitmask
 //                     for the tree tile), exchange the row maximum through shared memory,
 //                     and store their quarter of P (bf16 pairs) back into TMEM (tcgen05.st).
 //                     Four warps per SM sub-partition keep the exponential unit fed.  A
 //                     warp whose 32 rows are all padding only keeps the barriers.
-// S(t+1) and S(t+2) are computed while the softmax of tile t runs (three S and P buffers).  O lives in TMEM and is rescaled
-// lazily: only when a row's maximum grows by more than 2^8 over the reference the row's P
-// values were taken against (otherwise P <= 2^8, well inside bf16/fp32 range).  The last
-// split also runs the tree tile: its K/V rows come by TMA from a 4-D view of the tree K/V
-// ([B][N][Hkv][D], rows past N zero-filled) into the next ring slots.  Splits write (m, l,
-// acc) partials for the log-sum-exp merge; a single split normalises and writes the output.
+// S(t+1) is computed while the softmax of tile t runs (two S and two P buffers in TMEM).
+// O lives in TMEM and is rescaled lazily: only when a row's maximum grows by more than 2^8
+// over the reference the row's P values were taken against (otherwise P <= 2^8, well
+// inside bf16/fp32 range).  The last split also runs the tree tile: its K/V rows come by
+// TMA from a 4-D view of the tree K/V ([B][N][Hkv][D], rows past N zero-filled) into the
+// next ring slots.  Splits write (m, l, acc) partials for the log-sum-exp merge; a single
+// split normalises and writes the output.
 #pragma once
 
 #include "attention.cuh"
@@ -38,24 +40,20 @@ namespace eagle {
 constexpr int kTcRows = 128;  // MMA M: query rows per CTA
 constexpr int kTcSoftmaxWarps = 16;
 constexpr int kTcParts = kTcSoftmaxWarps / 4;       // warps sharing one TMEM lane quarter
-constexpr int kTcCols = 64 / kTcParts;              // score columns per softmax thread
-constexpr int kTcKWarp = kTcSoftmaxWarps;
+constexpr int kTcCols = kAttnKeys / kTcParts;       // score columns per softmax thread
+constexpr int kTcLoadWarp = kTcSoftmaxWarps;       // lane 0: Q and K tiles; lane 1: V tiles
 constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
-constexpr int kTcVWarp = kTcSoftmaxWarps + 2;
-constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 3);
+constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 2);
 constexpr float kTcRescaleThreshold = 8.0f;  // log2 units
 
-// Lite: the compact layout for a CTA that runs exactly one tile (one prefix tile, or the
-// tree tile in a CTA of its own): one K and one V slot.  It is small enough to share an SM
-// with two LM-head CTAs.
-template <int D, bool Lite = false>
+template <int D>
 struct TcSmem {
-  static constexpr int kKStages = Lite ? 1 : (D == 128 ? 6 : 8);
-  static constexpr int kVStages = Lite ? 1 : (D == 128 ? 5 : 8);
-  // S and P buffers in TMEM: three of each, so S(t + 2) can be computed while the softmax
-  // of tile t + 1 runs and the PV of tile t has not been issued yet
-  static constexpr int kSBufs = 3;
-  static constexpr int kTile = kAttnKeys * D * 2;  // one K or V tile (D/64 boxes of 64 x 128 B)
+  static constexpr int kKStages = D == 128 ? 3 : 5;
+  static constexpr int kVStages = D == 128 ? 2 : 5;
+  // S and P buffers in TMEM: two of each, so S(t + 1) is computed while the softmax of tile
+  // t runs
+  static constexpr int kSBufs = 2;
+  static constexpr int kTile = kAttnKeys * D * 2;  // one K or V tile (D/64 boxes of 128 x 128 B)
   static constexpr int kQ = kTcRows * D * 2;        // D/64 boxes of 128 rows x 128 B
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQ;
@@ -66,13 +64,13 @@ struct TcSmem {
   // exchange [part][row]
   static constexpr int kXchOff = kParOff + 64 * 4;
   static constexpr int kBarOff = kXchOff + 3 * kTcParts * kTcRows * 4;
-  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[3], s_free[3],
-  // p_full[3], pv_done[3], o_final
+  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], s_free[2],
+  // p_full[2], pv_done[2], o_final
   static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * kSBufs + 1;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  // TMEM columns: S0-S2 64 columns each [0, 192), O [192, 192 + D), P0-P2 32 columns each
-  // (64 bf16 per row, two to a column) after O
+  // TMEM columns: S0 / S1 128 columns each [0, 256), O [256, 256 + D), P0 / P1 64 columns
+  // each (128 bf16 per row, two to a column) after O
   static constexpr uint32_t kOCol = kSBufs * kAttnKeys;
   static constexpr uint32_t kPCol = kOCol + D;
   static constexpr uint32_t kTmemCols = 512;
@@ -83,12 +81,12 @@ struct TcAttnParams {
   int32_t nodes_per_block;  // NB: nodes per 128-row tile (G * NB <= 128)
 };
 
-template <int D, bool Lite = false>
+template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
                         const __grid_constant__ CUtensorMap tm_vt, const TcAttnParams tp) {
-  using SM = TcSmem<D, Lite>;
+  using SM = TcSmem<D>;
   constexpr int SK = SM::kKStages;
   constexpr int SV = SM::kVStages;
   const AttnParams& prm = tp.a;
@@ -125,14 +123,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int ntiles = (L + kAttnKeys - 1) / kAttnKeys;
   const int t_begin = split * prm.tiles_per_split;
   const int t_end = min(ntiles, t_begin + prm.tiles_per_split);
-  int nt = t_end > t_begin ? t_end - t_begin : 0;
-  bool last = split == prm.num_splits - 1;
-  if (Lite && nt + (last ? 1 : 0) > 1) {
-    // a plan that gives a compact-layout CTA two tiles: flag it and run nothing
-    if (threadIdx.x == 0) record_error(kErrAttnPlan);
-    nt = 0;
-    last = false;
-  }
+  const int nt = t_end > t_begin ? t_end - t_begin : 0;
+  const bool last = split == prm.num_splits - 1;
   const int T = nt + (last ? 1 : 0);  // tiles this CTA runs (prefix tiles, then the tree tile)
 
   if (threadIdx.x == 0) {
@@ -170,10 +162,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto k_stage = [&](int s) { return sbase + SM::kKOff + static_cast<uint32_t>(s) * SM::kTile; };
   auto v_stage = [&](int s) { return sbase + SM::kVOff + static_cast<uint32_t>(s) * SM::kTile; };
 
-  if (warp == kTcKWarp || warp == kTcVWarp) {
+  if (warp == kTcLoadWarp) {
     // ------------------------------------------------------------ TMA producers (K, V)
-    if (lane == 0) {
-      const bool is_k = warp == kTcKWarp;
+    if (lane < 2) {
+      const bool is_k = lane == 0;
       const int S = is_k ? SK : SV;
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
@@ -219,6 +211,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       auto issue_s = [&](int t) {
         const int s = t % SK, sb = t % NS;
         ok = ok && mbar_wait(smem_u32(&k_full[s]), (t / SK) & 1, kErrAttnMmaWait);
+        // buffer sb was last read (into registers) by the softmax of tile t - NS
         if (t >= NS) ok = ok && mbar_wait(smem_u32(&s_free[sb]), (t / NS - 1) & 1, kErrAttnMmaWait);
         tc_fence_after();
         const uint32_t kb = k_stage(s);
@@ -233,22 +226,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_commit(smem_u32(&s_full[sb]));
         tc_commit(smem_u32(&k_empty[s]));  // the K slot is free once S(t) has read it
       };
-      // S runs two tiles ahead of PV: S(t + 2) is queued as soon as its buffer and K tile
-      // are free, before PV(t) waits for the softmax of tile t
+      // S(t + 1) is queued before PV(t) waits for the softmax of tile t
       if (T > 0) issue_s(0);
-      if (T > 1) issue_s(1);
       for (int t = 0; t < T; ++t) {
-        if (t + 2 < T) issue_s(t + 2);
+        if (t + 1 < T) issue_s(t + 1);
         const int s = t % SV, pb = t % NS;
         ok = ok && mbar_wait(smem_u32(&p_full[pb]), (t / NS) & 1, kErrAttnMmaWait);
         ok = ok && mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnMmaWait);
         tc_fence_after();
         const uint32_t vb = v_stage(s);
-        const uint32_t pa = tmem + SM::kPCol + static_cast<uint32_t>(pb * 32);
+        const uint32_t pa = tmem + SM::kPCol + static_cast<uint32_t>(pb * (kAttnKeys / 2));
 #pragma unroll
         for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
           // 16 keys = 8 TMEM columns of P (bf16 pairs) and two 8-key groups of 1024 B of V;
-          // the second 64-column group of V is the next TMA box, one tile-half further
+          // the second 64-column group of V is the next TMA box, kAttnKeys x 128 B further
           const uint64_t bdesc = smem_desc_mn_sw128(vb + kk * 2048, kAttnKeys * 128, 1024);
           if (ok) tc_mma_f16_ts(o_tmem, pa + 8 * kk, bdesc, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
         }
@@ -296,8 +287,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     constexpr uint32_t kColMask = C == 32 ? 0xffffffffu : ((1u << C) - 1u);
     // this thread's C key columns of the tree tile, as a bit mask
-    const uint32_t tree_bits =
-        (last && rvalid) ? static_cast<uint32_t>(anc[node] >> (C * part)) & kColMask : 0u;
+    const uint32_t tree_bits = (last && rvalid && C * part < 64)
+                                   ? static_cast<uint32_t>(anc[node] >> (C * part)) & kColMask : 0u;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     float m_ref = -INFINITY, l = 0.f;
     for (int t = 0; t < T; ++t) {
@@ -357,12 +348,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_wait(smem_u32(&pv_done[(t - 1) % NS]), ((t - 1) / NS) & 1, kErrAttnConsumerWait);
           tc_fence_after();
           __syncwarp();
-          uint32_t ov[OC];
-          tmem_ld_cols<OC>(lane_base + SM::kOCol + OC * part, ov);
-          tmem_ld_wait();
+#pragma unroll 1
+          for (int c0 = 0; c0 < OC; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld_cols<16>(lane_base + SM::kOCol + OC * part + c0, ov);
+            tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < OC; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-          tmem_st_cols<OC>(lane_base + SM::kOCol + OC * part, ov);
+            for (int k = 0; k < 16; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+            tmem_st_cols<16>(lane_base + SM::kOCol + OC * part + c0, ov);
+          }
           tmem_st_wait();
         }
         if (rebase) {
@@ -373,7 +367,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // exp2(-inf) = 0 (and m = 0 while every key so far was masked)
         const float c = prm.scale_log2;
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-        // P buffer t % 3 was last read by PV(t - 3)
+        // P buffer t % 2 was last read by PV(t - 2)
         if (t >= NS) mbar_wait(smem_u32(&pv_done[sb]), (t / NS - 1) & 1, kErrAttnConsumerWait);
         uint32_t w[C / 2];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
@@ -388,7 +382,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         __syncwarp();
-        tmem_st_cols<C / 2>(lane_base + SM::kPCol + sb * 32 + (C / 2) * part, w);
+        tmem_st_cols<C / 2>(lane_base + SM::kPCol + sb * (kAttnKeys / 2) + (C / 2) * part, w);
         tmem_st_wait();
       }
       if (!tree) {
@@ -428,34 +422,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const bool single = prm.num_splits == 1;
     const float inv = (l > 0.f) ? 1.0f / l : 0.f;
     if (live) {
-      uint32_t ov[OC];
-      __syncwarp();  // the TMEM load below is warp-wide
-      if (T > 0) {
-        tmem_ld_cols<OC>(lane_base + SM::kOCol + OC * part, ov);
-        tmem_ld_wait();
-      } else {
+#pragma unroll 1
+      for (int cc = 0; cc < OC; cc += 16) {
+        uint32_t ov[16];
+        __syncwarp();  // the TMEM load below is warp-wide
+        if (T > 0) {
+          tmem_ld_cols<16>(lane_base + SM::kOCol + OC * part + cc, ov);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-        for (int k = 0; k < OC; ++k) ov[k] = 0u;
-      }
-      const int c0 = OC * part;
-      if (!rvalid) {
-      } else if (single) {
-        uint4* dst = reinterpret_cast<uint4*>(prm.out + prow_g * D + c0);
-#pragma unroll
-        for (int k = 0; k < OC; k += 8) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(ov[k + 2]) * inv, __uint_as_float(ov[k + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(ov[k + 4]) * inv, __uint_as_float(ov[k + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(ov[k + 6]) * inv, __uint_as_float(ov[k + 7]) * inv);
-          dst[k / 8] = w;
+          for (int k = 0; k < 16; ++k) ov[k] = 0u;
         }
-      } else {
-        float4* dst = reinterpret_cast<float4*>(prm.part_acc + (prow_g * prm.num_splits + split) * D + c0);
+        const int c0 = OC * part + cc;
+        if (!rvalid) {
+        } else if (single) {
+          uint4* dst = reinterpret_cast<uint4*>(prm.out + prow_g * D + c0);
 #pragma unroll
-        for (int k = 0; k < OC; k += 4)
-          dst[k / 4] = make_float4(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1]),
-                                   __uint_as_float(ov[k + 2]), __uint_as_float(ov[k + 3]));
+          for (int k = 0; k < 16; k += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ov[k + 2]) * inv, __uint_as_float(ov[k + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ov[k + 4]) * inv, __uint_as_float(ov[k + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ov[k + 6]) * inv, __uint_as_float(ov[k + 7]) * inv);
+            dst[k / 8] = w;
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(prm.part_acc + (prow_g * prm.num_splits + split) * D + c0);
+#pragma unroll
+          for (int k = 0; k < 16; k += 4)
+            dst[k / 4] = make_float4(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1]),
+                                     __uint_as_float(ov[k + 2]), __uint_as_float(ov[k + 3]));
+        }
       }
     }
     if (rvalid && !single && part == 0)

@@ -63,18 +63,12 @@ struct AttnPlan {
   int tiles_per_split;
   size_t acc_bytes;  // split partials (0 with a single split)
   size_t ml_bytes;
-  bool lite;         // one tile per CTA, compact shared-memory layout
 };
 
-// Split the prefix so that (sequences x kv heads x row blocks x splits) fills one wave of
-// one CTA per SM (the kernel's register use allows one); a split never spans more than 32
-// tiles of 64 keys.
-// `lite`: one tile per CTA (the compact shared-memory layout) -- every prefix tile is a
-// split of its own and the tree tile gets one more; used where the attention runs beside
-// the LM head rather than on an idle GPU.
-AttnPlan plan_attention(const eagle_shape_t* s, bool lite = false) {
+// Split the prefix so that (sequences x kv heads x row blocks x splits) runs in as few
+// waves of one CTA per SM as the work allows (the kernel's shared memory allows one).
+AttnPlan plan_attention(const eagle_shape_t* s) {
   AttnPlan p{};
-  p.lite = lite && s->dtype == EAGLE_DTYPE_BF16;
   const int G = s->num_q_heads / s->num_kv_heads;
   if (s->dtype == EAGLE_DTYPE_BF16) {
     // tensor-core path: a 128-row tile holds floor(128 / G) nodes x G heads
@@ -85,17 +79,9 @@ AttnPlan plan_attention(const eagle_shape_t* s, bool lite = false) {
     p.row_blocks = 1;
   }
   const int max_tiles = (s->max_prefix_len + kAttnKeys - 1) / kAttnKeys;
-  if (p.lite) {
-    p.tiles_per_split = 1;
-    p.splits = max_tiles + 1;
-    const size_t rows = static_cast<size_t>(s->batch) * s->num_nodes * s->num_q_heads;
-    p.acc_bytes = align256(rows * p.splits * s->head_dim * sizeof(float));
-    p.ml_bytes = align256(rows * p.splits * 2 * sizeof(float));
-    return p;
-  }
-  // one CTA per SM at a time: pick the split count that minimises waves x (tiles per split
-  // + a CTA's fixed cost, about four tiles' time: set-up, pipeline fill, the tree tile, the
-  // partials it writes for the merge)
+  // pick the split count that minimises waves x (tiles per split + a CTA's fixed cost,
+  // about two tiles' time: set-up, pipeline fill, the tree tile, the partials it writes
+  // for the merge)
   const long base = static_cast<long>(s->batch) * s->num_kv_heads * p.row_blocks;
   int best_splits = 1;
   long best_cost = -1;
@@ -103,7 +89,7 @@ AttnPlan plan_attention(const eagle_shape_t* s, bool lite = false) {
     const long tiles_per = max_tiles > 0 ? (max_tiles + sp - 1) / sp : 0;
     if (sp > 1 && (tiles_per - 1) * sp >= max_tiles) continue;  // same split count as a smaller sp
     const long waves = (base * sp + kNumSMs - 1) / kNumSMs;
-    const long cost = waves * (tiles_per + 4);
+    const long cost = waves * (tiles_per + 2);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best_splits = sp;
@@ -183,40 +169,11 @@ AccPlan plan_accept(const eagle_shape_t* s, int max_cluster = kAccMaxCluster) {
 
 constexpr size_t kAccMaxSmem = kAccSmemBudget;
 
-// ------------------------------------------------------------------ the step's schedule
+// ------------------------------------------------------------------ workspace
 
-// eagle_verify_step runs tree attention beside the LM head when both fit on one SM at
-// once: with a 3-stage ring the LM head (HBM-bound, two CTAs per SM) leaves room for one
-// compact-layout attention CTA, so the attention hides under the weight stream instead of
-// running after it.  Only for a single chunk of tree rows, and while the one-tile-per-CTA
-// partials stay modest.
-constexpr int kStepLmStages = 3;
-constexpr size_t kSmemPerSM = 228 * 1024;
-constexpr size_t kSmemPerCtaReserve = 1024;
-constexpr size_t kMaxOverlapWorkspace = 256ull << 20;
-
-size_t attention_ws_bytes(const eagle_shape_t* s, bool lite) {
-  const AttnPlan p = plan_attention(s, lite);
+size_t attention_ws_bytes(const eagle_shape_t* s) {
+  const AttnPlan p = plan_attention(s);
   return p.acc_bytes + p.ml_bytes;
-}
-
-bool step_overlap(const eagle_shape_t* s);
-
-// the attention partials' share of the workspace: enough for either plan the step may take
-size_t attention_region_bytes(const eagle_shape_t* s) {
-  const size_t alone = attention_ws_bytes(s, false);
-  if (!step_overlap(s)) return alone;
-  const size_t beside = attention_ws_bytes(s, true);
-  return beside > alone ? beside : alone;
-}
-
-bool step_overlap(const eagle_shape_t* s) {
-  if (s->dtype != EAGLE_DTYPE_BF16) return false;
-  const LmPlan lm = plan_lm_head(s, kStepLmStages);
-  if (lm.chunks != 1) return false;
-  const size_t attn = s->head_dim == 64 ? TcSmem<64, true>::kAlloc : TcSmem<128, true>::kAlloc;
-  if (2 * (lm.smem + kSmemPerCtaReserve) + attn + kSmemPerCtaReserve > kSmemPerSM) return false;
-  return attention_ws_bytes(s, true) <= kMaxOverlapWorkspace;
 }
 
 // ------------------------------------------------------------------ driver entry point
@@ -256,7 +213,7 @@ struct DeviceState {
   std::once_flag side_once;
   bool side_ok = false;
   cudaStream_t side = nullptr;
-  cudaEvent_t lm_mark = nullptr;  // LM head under way (T = 0 beside it) or completed
+  cudaEvent_t lm_mark = nullptr;  // LM head completed
   cudaEvent_t attn_done = nullptr;
   std::mutex step_mu;  // one step's fork/join sequence at a time on the shared side stream
   // eagle_draft_select: shared-memory limits set once; clusters of S CTAs resident at once,
@@ -286,10 +243,6 @@ bool ensure_attributes(int dev) {
                                TcSmem<64>::kAlloc) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TcSmem<128>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               TcSmem<64, true>::kAlloc) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               TcSmem<128, true>::kAlloc) == cudaSuccess;
     const void* walks[2] = {reinterpret_cast<const void*>(tree_accept_kernel<true>),
                             reinterpret_cast<const void*>(tree_accept_kernel<false>)};
     bool nonportable = true;
@@ -339,11 +292,9 @@ eagle_status_t launch_status() {
 
 // ------------------------------------------------------------------ launches
 
-// `lite`: the one-tile-per-CTA plan and compact layout (the step's greedy schedule).
 eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* kp, const void* vp,
                              const int32_t* lens, const void* kt, const void* vt,
-                             const int32_t* parents, void* out, void* ws, cudaStream_t st,
-                             bool lite = false) {
+                             const int32_t* parents, void* out, void* ws, cudaStream_t st) {
   const int B = s->batch, N = s->num_nodes, Hq = s->num_q_heads, Hkv = s->num_kv_heads;
   const int D = s->head_dim, Lmax = s->max_prefix_len;
   const float scale = softmax_scale(s);
@@ -362,7 +313,7 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
           N, Hq, Hkv, Lmax, scale);
     return launch_status();
   }
-  const AttnPlan plan = plan_attention(s, lite);
+  const AttnPlan plan = plan_attention(s);
   const int G = Hq / Hkv;
   CUtensorMap tq, tk, tv, tkt, tvt;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Lmax),
@@ -408,16 +359,11 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(plan.row_blocks, plan.splits, B * Hkv);
   cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = plan.lite ? (D == 64 ? TcSmem<64, true>::kAlloc : TcSmem<128, true>::kAlloc)
-                                   : (D == 64 ? TcSmem<64>::kAlloc : TcSmem<128>::kAlloc);
+  cfg.dynamicSmemBytes = D == 64 ? TcSmem<64>::kAlloc : TcSmem<128>::kAlloc;
   cfg.stream = st;
   cudaError_t e;
-  if (plan.lite)
-    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64, true>, tq, tk, tv, tkt, tvt, tp)
-                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128, true>, tq, tk, tv, tkt, tvt, tp);
-  else
-    e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, tq, tk, tv, tkt, tvt, tp)
-                : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, tq, tk, tv, tkt, tvt, tp);
+  e = D == 64 ? cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<64>, tq, tk, tv, tkt, tvt, tp)
+              : cudaLaunchKernelEx(&cfg, tree_attn_tc_kernel<128>, tq, tk, tv, tkt, tvt, tp);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return EAGLE_ERR_CUDA;
@@ -458,10 +404,8 @@ eagle_status_t run_lm_head_persistent(const eagle_shape_t* s, const void* hidden
   return launch_status();
 }
 
-// `started`: an event that fires once every CTA has begun (the LM head's resources are
-// claimed), for a second stream to start work beside it; `max_stages` caps the TMA ring.
 eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const void* w, float* logits,
-                           cudaStream_t st, int max_stages = 8, cudaEvent_t started = nullptr) {
+                           cudaStream_t st) {
   const int M = s->batch * s->num_nodes, V = s->vocab, H = s->hidden;
   if (s->dtype == EAGLE_DTYPE_F32) {
     const dim3 grid((V + kLmF32TileV - 1) / kLmF32TileV, (M + kLmF32TileR - 1) / kLmF32TileR);
@@ -469,8 +413,8 @@ eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const voi
                                              logits, M, V, H);
     return launch_status();
   }
-  const LmPlan plan = plan_lm_head(s, max_stages);
-  if (plan.chunks > 1 && started == nullptr) return run_lm_head_persistent(s, hidden, w, logits, st, plan);
+  const LmPlan plan = plan_lm_head(s);
+  if (plan.chunks > 1) return run_lm_head_persistent(s, hidden, w, logits, st, plan);
   CUtensorMap tw, th;
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(V)};
   const cuuint64_t hd[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(M)};
@@ -481,25 +425,6 @@ eagle_status_t run_lm_head(const eagle_shape_t* s, const void* hidden, const voi
     return EAGLE_ERR_CUDA;
   LmTcParams prm{logits, M, V, H, plan.bn, plan.stages, plan.tmem_cols};
   const dim3 grid(plan.chunks, (V + kLmBlockV - 1) / kLmBlockV);
-  if (started != nullptr) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kLmThreads);
-    cfg.dynamicSmemBytes = plan.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeLaunchCompletionEvent;
-    attr[0].val.launchCompletionEvent.event = started;
-    attr[0].val.launchCompletionEvent.flags = 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, lm_head_tc_kernel, tw, th, prm) == cudaSuccess) return launch_status();
-    // no launch-completion events here: the second stream starts after the LM head instead
-    cudaGetLastError();
-    lm_head_tc_kernel<<<grid, kLmThreads, plan.smem, st>>>(tw, th, prm);
-    if (cudaEventRecord(started, st) != cudaSuccess) return EAGLE_ERR_CUDA;
-    return launch_status();
-  }
   lm_head_tc_kernel<<<grid, kLmThreads, plan.smem, st>>>(tw, th, prm);
   return launch_status();
 }
@@ -794,7 +719,7 @@ const char* eagle_status_string(eagle_status_t status) {
 
 size_t eagle_workspace_bytes(const eagle_shape_t* shape) {
   if (check_shape(shape) != EAGLE_OK) return 0;
-  return attention_region_bytes(shape);
+  return attention_ws_bytes(shape);
 }
 
 eagle_status_t eagle_tree_attention(const eagle_shape_t* shape, const void* q, const void* k_prefix,
@@ -861,23 +786,17 @@ eagle_status_t eagle_verify_step(const eagle_shape_t* shape, const void* q, cons
     // Two streams.  The LM head streams W over the whole GPU and the accept walk follows it
     // on the caller's stream (programmatic dependent launch: the walk's set-up overlaps the
     // LM head's drain).  Tree attention, whose output the walk does not read, runs with its
-    // merge on a library-owned side stream, and the caller's stream waits for it after the
-    // walk.  Greedy steps on shapes with few tree rows start it beside the LM head (compact
-    // layout, one tile per CTA) once every LM-head CTA holds its SM: there the walk is one
-    // argmax per accepted node and the attention would be the step's tail.  Otherwise it
-    // starts when the LM head completes and runs while the walk runs.  No kernel is ever
-    // launched as a programmatic dependent of the walk.
+    // merge on a library-owned side stream once the LM head has completed, beside the walk,
+    // and the caller's stream waits for it after the walk.  No kernel is ever launched as a
+    // programmatic dependent of the walk.
     DeviceState& ds = g_dev[dev];
     std::lock_guard<std::mutex> lock(ds.step_mu);
-    const bool beside = temperature == 0.f && step_overlap(shape) &&
-                        workspace_bytes >= attention_ws_bytes(shape, true);
-    rc = run_lm_head(shape, hidden, w_lm, logits, st, beside ? kStepLmStages : 8,
-                     beside ? ds.lm_mark : nullptr);
+    rc = run_lm_head(shape, hidden, w_lm, logits, st);
     if (rc != EAGLE_OK) return rc;
-    if (!beside && cudaEventRecord(ds.lm_mark, st) != cudaSuccess) return EAGLE_ERR_CUDA;
+    if (cudaEventRecord(ds.lm_mark, st) != cudaSuccess) return EAGLE_ERR_CUDA;
     if (cudaStreamWaitEvent(ds.side, ds.lm_mark, 0) != cudaSuccess) return EAGLE_ERR_CUDA;
     rc = run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,
-                       workspace, ds.side, /*lite=*/beside);
+                       workspace, ds.side);
     if (rc != EAGLE_OK) return rc;
     if (cudaEventRecord(ds.attn_done, ds.side) != cudaSuccess) return EAGLE_ERR_CUDA;
     rc = run_accept(shape, logits, draft_probs, tokens, parents, temperature, seed, offset,
@@ -1023,14 +942,14 @@ extern "C" eagle_status_t eagle_tree_attention_static(const eagle_shape_t* shape
                                                       const void* v_tree, const int32_t* parents,
                                                       void* out, void* stream) {
   if (check_shape(shape) != EAGLE_OK) return EAGLE_ERR_INVALID_ARGUMENT;
-  if (attention_ws_bytes(shape, false) > EAGLE_STATIC_SCRATCH_BYTES) return EAGLE_ERR_UNSUPPORTED;
+  if (attention_ws_bytes(shape) > EAGLE_STATIC_SCRATCH_BYTES) return EAGLE_ERR_UNSUPPORTED;
   int dev;
   if (!current_device(&dev)) return EAGLE_ERR_CUDA;
   void* scratch = static_scratch_address(dev);
   if (scratch == nullptr) return EAGLE_ERR_CUDA;
   eagle_status_t rc = check_attention_args(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree,
                                            parents, out, scratch, EAGLE_STATIC_SCRATCH_BYTES,
-                                           attention_ws_bytes(shape, false));
+                                           attention_ws_bytes(shape));
   if (rc != EAGLE_OK) return rc;
   if (!ensure_attributes(dev)) return EAGLE_ERR_CUDA;
   return run_attention(shape, q, k_prefix, v_prefix, prefix_lens, k_tree, v_tree, parents, out,

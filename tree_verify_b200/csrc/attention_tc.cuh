@@ -7,29 +7,32 @@
 // r -> node i0 + r / G, head kvh*G + r % G), so one 128-row MMA tile covers all of them and
 // every prefix K/V tile is read from HBM once.
 //
-//   warp 16 lane 0    TMA: the Q tile once (a 3-D box over [B*N, Hq, D]) and the 128-key K
-//                     tiles of this split into the K ring;
-//   warp 16 lane 1    TMA: the matching V tiles into the V ring (its own ring and barriers,
-//                     so a K slot is refilled as soon as S = Q K^T has read it, a tile
-//                     earlier than its V slot);
-//   warp 17 (lane 0)  tcgen05.mma: S = Q K^T (M 128, N 128, K = D) into one of two TMEM
-//                     buffers, then O += P V (M 128, N = D, K 128) with P read from TMEM and
-//                     V as an MN-major operand straight from its TMA tile (128-key tiles:
-//                     fewer, larger MMA instructions per key);
-//   warps 0-15        four threads per query row (= TMEM lane): warps w, w + 4, w + 8 and
-//                     w + 12 share the lane quarter w % 4 and take 32 of the tile's 128 scores
-//                     each (tcgen05.ld), mask them (prefix length, or the ancestor bitmask
-//                     for the tree tile), exchange the row maximum through shared memory,
-//                     and store their quarter of P (bf16 pairs) back into TMEM (tcgen05.st).
-//                     Four warps per SM sub-partition keep the exponential unit fed.  A
-//                     warp whose 32 rows are all padding only keeps the barriers.
-// S(t+1) is computed while the softmax of tile t runs (two S and two P buffers in TMEM).
-// O lives in TMEM and is rescaled lazily: only when a row's maximum grows by more than 2^8
-// over the reference the row's P values were taken against (otherwise P <= 2^8, well
-// inside bf16/fp32 range).  The last split also runs the tree tile: its K/V rows come by
-// TMA from a 4-D view of the tree K/V ([B][N][Hkv][D], rows past N zero-filled) into the
-// next ring slots.  Splits write (m, l, acc) partials for the log-sum-exp merge; a single
-// split normalises and writes the output.
+// Keys arrive in tiles of 128 (one TMA box per 64 columns of D).  Each tile is split
+// between two softmax groups: group 0 takes keys 0-63 of every tile, group 1 keys 64-127.
+// A group keeps its own running maximum, denominator and output accumulator O_g, so the
+// two groups never wait for each other: while one exponentiates (SFU and FMA pipes), the
+// other loads scores and takes maxima, and the tensor core runs the other group's MMAs.
+// The two partial results are merged by log-sum-exp at the end.
+//
+//   warps 0-3 / 4-7   softmax groups 0 / 1: one thread per query row (TMEM lane = row,
+//                     warp w serves lane quarter w % 4): tcgen05.ld of the group's 64
+//                     scores, mask (prefix length, or the ancestor bitmask on the tree
+//                     tile), row maximum, P = 2^(s * c - m), tcgen05.st of P (bf16 pairs);
+//   warp 8 lane 0     TMA: the Q tile once (a 3-D box over [B*N, Hq, D]), then the K tiles;
+//   warp 8 lane 1     TMA: the V tiles (their own ring, so a K slot refills as soon as both
+//                     S MMAs have read it, ahead of its V slot);
+//   warp 9 lane 0     tcgen05.mma: S_g = Q K_g^T (M 128, N 64, K = D) and O_g += P_g V_g
+//                     (M 128, N = D, K 64; P read from TMEM, V an MN-major operand straight
+//                     from its TMA tile);
+//   warps 10-11       no role (a 384-thread block caps registers at 168, which three warps
+//                     per SM sub-partition can hold).
+// TMEM: S_0 S_1 (64 columns each), P_0 P_1 (32), O_0 O_1 (D each).  O_g is rescaled lazily,
+// only when the group's row maximum grows by more than 2^8 over the reference its P values
+// were taken against.  A commit on s_full_g(t) covers every earlier MMA, PV_g(t-1) included,
+// so a group that sees S_g(t) may overwrite P_g and rescale O_g.  The last split also runs
+// the tree tile: its K/V rows come by TMA from a 4-D view of the tree K/V ([B][N][Hkv][D],
+// rows past N zero-filled).  Splits write (m, l, acc) partials for the log-sum-exp merge; a
+// single split normalises and writes the output.
 #pragma once
 
 #include "attention.cuh"
@@ -37,22 +40,22 @@
 
 namespace eagle {
 
-constexpr int kTcRows = 128;  // MMA M: query rows per CTA
-constexpr int kTcSoftmaxWarps = 16;
-constexpr int kTcParts = kTcSoftmaxWarps / 4;       // warps sharing one TMEM lane quarter
-constexpr int kTcCols = kAttnKeys / kTcParts;       // score columns per softmax thread
-constexpr int kTcLoadWarp = kTcSoftmaxWarps;       // lane 0: Q and K tiles; lane 1: V tiles
-constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
-constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 2);
-constexpr float kTcRescaleThreshold = 8.0f;  // log2 units
+constexpr int kTcRows = 128;                  // MMA M: query rows per CTA
+constexpr int kTcHalf = kAttnKeys / 2;        // keys of a tile per softmax group
+constexpr int kTcSoftmaxWarps = 8;            // two groups of four
+constexpr int kTcLoadWarp = 8;                // lane 0: Q and K tiles; lane 1: V tiles
+constexpr int kTcMmaWarp = 9;
+constexpr int kTcThreads = 32 * 12;
+constexpr float kTcRescaleThreshold = 8.0f;   // log2 units
+// Of every 8 pairs of scores a softmax thread exponentiates, this many go through the
+// polynomial 2^x on the FMA pipe (exp2_poly2) and the rest through the SFU, whose 16
+// results per clock per SM would otherwise bound the softmax.
+constexpr int kTcPolyPairs = 2;
 
 template <int D>
 struct TcSmem {
   static constexpr int kKStages = D == 128 ? 3 : 5;
   static constexpr int kVStages = D == 128 ? 2 : 5;
-  // S and P buffers in TMEM: two of each, so S(t + 1) is computed while the softmax of tile
-  // t runs
-  static constexpr int kSBufs = 2;
   static constexpr int kTile = kAttnKeys * D * 2;  // one K or V tile (D/64 boxes of 128 x 128 B)
   static constexpr int kQ = kTcRows * D * 2;        // D/64 boxes of 128 rows x 128 B
   static constexpr int kQOff = 0;
@@ -60,19 +63,17 @@ struct TcSmem {
   static constexpr int kVOff = kKOff + kKStages * kTile;
   static constexpr int kAncOff = kVOff + kVStages * kTile;
   static constexpr int kParOff = kAncOff + 64 * 8;
-  // row-maximum exchange [tile parity][part][row] and, after the loop, the denominator
-  // exchange [part][row]
+  // the groups' (m, l) per row for the final merge: [group][2][row]
   static constexpr int kXchOff = kParOff + 64 * 4;
-  static constexpr int kBarOff = kXchOff + 3 * kTcParts * kTcRows * 4;
-  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], s_free[2],
-  // p_full[2], pv_done[2], o_final
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * kSBufs + 1;
+  static constexpr int kBarOff = kXchOff + 2 * 2 * kTcRows * 4;
+  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], p_full[2], o_final
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 1;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  // TMEM columns: S0 / S1 128 columns each [0, 256), O [256, 256 + D), P0 / P1 64 columns
-  // each (128 bf16 per row, two to a column) after O
-  static constexpr uint32_t kOCol = kSBufs * kAttnKeys;
-  static constexpr uint32_t kPCol = kOCol + D;
+  // TMEM columns
+  static constexpr uint32_t kSCol = 0;                  // S_g at kSCol + 64 g
+  static constexpr uint32_t kPCol = 2 * kTcHalf;        // P_g at kPCol + 32 g
+  static constexpr uint32_t kOCol = 256;                // O_g at kOCol + D g
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -96,18 +97,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   uint64_t* anc = reinterpret_cast<uint64_t*>(smem + SM::kAncOff);
   int32_t* par_s = reinterpret_cast<int32_t*>(smem + SM::kParOff);
+  float* xch = reinterpret_cast<float*>(smem + SM::kXchOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
   uint64_t* q_full = bars;
   uint64_t* k_full = q_full + 1;
   uint64_t* k_empty = k_full + SK;
   uint64_t* v_full = k_empty + SK;
   uint64_t* v_empty = v_full + SV;
-  constexpr int NS = SM::kSBufs;
-  uint64_t* s_full = v_empty + SV;
-  uint64_t* s_free = s_full + NS;
-  uint64_t* p_full = s_free + NS;
-  uint64_t* pv_done = p_full + NS;
-  uint64_t* o_final = pv_done + NS;
+  uint64_t* s_full = v_empty + SV;  // [group]
+  uint64_t* p_full = s_full + 2;    // [group]
+  uint64_t* o_final = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -140,11 +139,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
     }
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_free[i]), 32 * kTcSoftmaxWarps);
-      mbar_init(smem_u32(&p_full[i]), 32 * kTcSoftmaxWarps);
-      mbar_init(smem_u32(&pv_done[i]), 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(smem_u32(&s_full[g]), 1);
+      mbar_init(smem_u32(&p_full[g]), 4);  // one arrival per warp of the group
     }
     mbar_init(smem_u32(o_final), 1);
     fence_mbar_init();
@@ -190,7 +187,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int h = 0; h < D / 64; ++h) tma_load_3d(dst + h * kAttnKeys * 128, map, fb, h * 64, key0, bk);
         } else {
-          // the tree tile: nodes 0..63 of (b, kvh); nodes past N are zero-filled
+          // the tree tile: nodes 0..127 of (b, kvh); nodes past N are zero-filled
 #pragma unroll
           for (int h = 0; h < D / 64; ++h) tma_load_4d(dst + h * kAttnKeys * 128, tmap, fb, h * 64, kvh, 0, b);
         }
@@ -204,18 +201,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == kTcMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kTcRows, kAttnKeys);
+      const uint32_t idesc_s = idesc_bf16_f32(kTcRows, kTcHalf);
       const uint32_t idesc_o = idesc_bf16_f32_bmn(kTcRows, D);
-      const uint32_t o_tmem = tmem + SM::kOCol;
       bool ok = mbar_wait(smem_u32(q_full), 0, kErrAttnMmaWait);
-      auto issue_s = [&](int t) {
-        const int s = t % SK, sb = t % NS;
-        ok = ok && mbar_wait(smem_u32(&k_full[s]), (t / SK) & 1, kErrAttnMmaWait);
-        // buffer sb was last read (into registers) by the softmax of tile t - NS
-        if (t >= NS) ok = ok && mbar_wait(smem_u32(&s_free[sb]), (t / NS - 1) & 1, kErrAttnMmaWait);
+      // S_g(t) = Q K^T over keys [64 g, 64 g + 64) of tile t.  Buffer S_g was last read by
+      // the group's softmax of tile t - 1, which finished before its p_full arrival, and
+      // that was waited for before PV_g(t - 1) was issued.
+      auto issue_s = [&](int t, int g) {
+        const int s = t % SK;
+        if (g == 0) ok = ok && mbar_wait(smem_u32(&k_full[s]), (t / SK) & 1, kErrAttnMmaWait);
         tc_fence_after();
-        const uint32_t kb = k_stage(s);
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(sb * kAttnKeys);
+        const uint32_t kb = k_stage(s) + static_cast<uint32_t>(g * kTcHalf * 128);
+        const uint32_t d_tmem = tmem + SM::kSCol + static_cast<uint32_t>(g * kTcHalf);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int h = kk >> 2, k4 = kk & 3;
@@ -223,52 +220,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t bdesc = smem_desc_k_sw128(kb + h * kAttnKeys * 128) + 2 * k4;
           if (ok) tc_mma_f16(d_tmem, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[sb]));
-        tc_commit(smem_u32(&k_empty[s]));  // the K slot is free once S(t) has read it
+        tc_commit(smem_u32(&s_full[g]));
+        if (g == 1) tc_commit(smem_u32(&k_empty[s]));  // both halves of the K slot are read
       };
-      // S(t + 1) is queued before PV(t) waits for the softmax of tile t
-      if (T > 0) issue_s(0);
-      for (int t = 0; t < T; ++t) {
-        if (t + 1 < T) issue_s(t + 1);
-        const int s = t % SV, pb = t % NS;
-        ok = ok && mbar_wait(smem_u32(&p_full[pb]), (t / NS) & 1, kErrAttnMmaWait);
-        ok = ok && mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnMmaWait);
+      // O_g += P_g V over the group's 64 keys: 4 MMAs of 16 keys (8 TMEM columns of P, two
+      // 8-key groups of 1024 B of V; the second 64-column group of V is the next TMA box)
+      auto issue_pv = [&](int t, int g) {
+        const int s = t % SV;
+        ok = ok && mbar_wait(smem_u32(&p_full[g]), t & 1, kErrAttnMmaWait);
+        if (g == 0) ok = ok && mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnMmaWait);
         tc_fence_after();
-        const uint32_t vb = v_stage(s);
-        const uint32_t pa = tmem + SM::kPCol + static_cast<uint32_t>(pb * (kAttnKeys / 2));
+        const uint32_t vb = v_stage(s) + static_cast<uint32_t>(g * kTcHalf * 128);
+        const uint32_t pa = tmem + SM::kPCol + static_cast<uint32_t>(g * (kTcHalf / 2));
+        const uint32_t o_tmem = tmem + SM::kOCol + static_cast<uint32_t>(g * D);
 #pragma unroll
-        for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
-          // 16 keys = 8 TMEM columns of P (bf16 pairs) and two 8-key groups of 1024 B of V;
-          // the second 64-column group of V is the next TMA box, kAttnKeys x 128 B further
+        for (int kk = 0; kk < kTcHalf / 16; ++kk) {
           const uint64_t bdesc = smem_desc_mn_sw128(vb + kk * 2048, kAttnKeys * 128, 1024);
           if (ok) tc_mma_f16_ts(o_tmem, pa + 8 * kk, bdesc, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(smem_u32(&pv_done[pb]));
-        tc_commit(smem_u32(&v_empty[s]));
+        if (g == 1) tc_commit(smem_u32(&v_empty[s]));
+      };
+      if (T > 0) {
+        issue_s(0, 0);
+        issue_s(0, 1);
+      }
+      for (int t = 0; t < T; ++t) {
+        issue_pv(t, 0);
+        if (t + 1 < T) issue_s(t + 1, 0);
+        issue_pv(t, 1);
+        if (t + 1 < T) issue_s(t + 1, 1);
       }
       tc_commit(smem_u32(o_final));
     }
-  } else {
-    // ------------------------------------------------------------ softmax warps
-    constexpr int kSoftThreads = 32 * kTcSoftmaxWarps;
-    constexpr int C = kTcCols;              // score columns of this thread
-    constexpr int OC = D / kTcParts;        // output columns of this thread
+  } else if (warp < kTcSoftmaxWarps) {
+    // ------------------------------------------------------------ softmax groups
+    const int grp = warp >> 2;              // keys [64 grp, 64 grp + 64) of every tile
     const int quarter = warp & 3;           // TMEM lane quarter = row block of 32
-    const int part = warp >> 2;             // which C of the 64 scores, which OC of O
     const int r = quarter * 32 + lane;      // query row = TMEM lane
     const int node = i0 + r / G;
     const int head = kvh * G + r % G;
     const bool rvalid = r < rows_blk && node < N;
     // a warp with no real row skips the score and output work (its rows of P and O are
-    // never read for an output), but keeps every barrier; the warps of a quarter cover the
-    // same rows, so they are live together
+    // never read for an output), but keeps every barrier
     const bool live = __any_sync(0xffffffffu, rvalid);
-    const int tid = threadIdx.x;            // 0 .. kSoftThreads-1
-    float* xch = reinterpret_cast<float*>(smem + SM::kXchOff);
-    const uint32_t quarter_bar = 2 + quarter;  // named barrier of the warps sharing a quarter
-    auto quarter_sync = [&]() {
-      asm volatile("bar.sync %0, %1;" ::"r"(quarter_bar), "r"(32 * kTcParts) : "memory");
-    };
+    const int tid = threadIdx.x;            // 0 .. 255
+    constexpr int kSoftThreads = 32 * kTcSoftmaxWarps;
     if (last) {
       if (tid < N) {
         // ancestor bitmask: node tid and every node up its parent chain (a link that does
@@ -285,77 +281,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // named barrier of the softmax warps: the masks are read below
       asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
     }
-    constexpr uint32_t kColMask = C == 32 ? 0xffffffffu : ((1u << C) - 1u);
-    // this thread's C key columns of the tree tile, as a bit mask
-    const uint32_t tree_bits = (last && rvalid && C * part < 64)
-                                   ? static_cast<uint32_t>(anc[node] >> (C * part)) & kColMask : 0u;
+    // the tree keys are nodes 0..N-1 <= 63: all in group 0's half of the tree tile
+    const uint64_t tree_bits = (last && rvalid && grp == 0) ? anc[node] : 0ull;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t s_col = lane_base + SM::kSCol + static_cast<uint32_t>(grp * kTcHalf);
+    const uint32_t p_col = lane_base + SM::kPCol + static_cast<uint32_t>(grp * (kTcHalf / 2));
+    const uint32_t o_col = lane_base + SM::kOCol + static_cast<uint32_t>(grp * D);
+    const float c = prm.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     for (int t = 0; t < T; ++t) {
       const bool tree = t >= nt;
-      const int sb = t % NS;
-      mbar_wait(smem_u32(&s_full[sb]), (t / NS) & 1, kErrAttnConsumerWait);
+      mbar_wait(smem_u32(&s_full[grp]), t & 1, kErrAttnConsumerWait);
       tc_fence_after();
-      uint32_t sv[C];
       if (live) {
-        __syncwarp();  // the TMEM load below is warp-wide
-        tmem_ld_cols<C>(lane_base + sb * kAttnKeys + C * part, sv);
+        uint32_t sa[32], sb[32];
+        __syncwarp();  // the TMEM loads below are warp-wide
+        tmem_ld_cols<32>(s_col, sa);
+        tmem_ld_cols<32>(s_col + 32, sb);
         tmem_ld_wait();
-      }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[sb]));
-      if (live) {
-        // visibility of this thread's C keys
+        // visibility of this group's 64 keys
         const int first = tree ? 0 : (t_begin + t) * kAttnKeys;
-        const int valid = (tree ? N : min(kAttnKeys, L - first)) - C * part;
-        uint32_t vis = valid >= C ? kColMask : (valid <= 0 ? 0u : ((1u << valid) - 1u));
+        const int valid = (tree ? N : min(kAttnKeys, L - first)) - grp * kTcHalf;
+        uint64_t vis = valid >= kTcHalf ? ~0ull : (valid <= 0 ? 0ull : ((1ull << valid) - 1ull));
         if (tree) vis &= tree_bits;
-        if (!rvalid) vis = 0u;
+        if (!rvalid) vis = 0ull;
         // raw scores; masked ones (past L_b, outside the ancestor set, padding rows) become
         // -inf, which also drops any non-finite value the padding holds
-        float x[C];
+        float x[kTcHalf];
 #pragma unroll
-        for (int j = 0; j < C; ++j) x[j] = __uint_as_float(sv[j]);
-        if (vis != kColMask) {
-#pragma unroll
-          for (int j = 0; j < C; ++j) x[j] = ((vis >> j) & 1u) ? x[j] : -INFINITY;
+        for (int j = 0; j < 32; ++j) {
+          x[j] = __uint_as_float(sa[j]);
+          x[j + 32] = __uint_as_float(sb[j]);
         }
-        // tile maximum by a tree (short dependency chains)
-        float mx[C / 4];
+        if (vis != ~0ull) {
 #pragma unroll
-        for (int j = 0; j < C / 4; ++j)
-          mx[j] = fmaxf(fmaxf(x[j], x[j + C / 4]), fmaxf(x[j + C / 2], x[j + 3 * C / 4]));
+          for (int j = 0; j < kTcHalf; ++j) x[j] = ((vis >> j) & 1ull) ? x[j] : -INFINITY;
+        }
+        // row maximum by a tree of three-input maxima (32 instructions for 64 values)
+        float m3[22];
 #pragma unroll
-        for (int w2 = C / 8; w2 >= 1; w2 >>= 1)
+        for (int j = 0; j < 21; ++j) m3[j] = fmax3f(x[3 * j], x[3 * j + 1], x[3 * j + 2]);
+        m3[21] = x[63];
+        float n3[8];
 #pragma unroll
-          for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-        float tmax = mx[0];
-        // row maximum of the tile: combine with the other parts of the row; in scaled log2
-        // units (the scale is positive, so the maximum commutes with it)
-        xch[((t & 1) * kTcParts + part) * kTcRows + r] = tmax;
-        quarter_sync();
-#pragma unroll
-        for (int o = 1; o < kTcParts; ++o)
-          tmax = fmaxf(tmax, xch[((t & 1) * kTcParts + ((part + o) % kTcParts)) * kTcRows + r]);
-        tmax *= prm.scale_log2;
+        for (int j = 0; j < 7; ++j) n3[j] = fmax3f(m3[3 * j], m3[3 * j + 1], m3[3 * j + 2]);
+        n3[7] = m3[21];
+        // in scaled log2 units (the scale is positive, so the maximum commutes with it)
+        const float tmax =
+            fmax3f(fmax3f(n3[0], n3[1], n3[2]), fmax3f(n3[3], n3[4], n3[5]), fmaxf(n3[6], n3[7])) * c;
         const float m_new = fmaxf(m_ref, tmax);
         const bool rebase =
             m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kTcRescaleThreshold);
-        const bool scale_o = rebase && m_ref != -INFINITY;  // O holds P V taken against m_ref
+        const bool scale_o = rebase && m_ref != -INFINITY;  // O_g holds P V taken against m_ref
         const float f = scale_o ? fast_exp2(m_ref - m_new) : 1.0f;
-        // TMEM loads/stores are warp-wide: the warp rescales if any of its rows must
+        // TMEM loads/stores are warp-wide: the warp rescales if any of its rows must.
+        // PV_g(t - 1) is complete: s_full_g(t) was committed after it.
         if (__any_sync(0xffffffffu, scale_o)) {
-          mbar_wait(smem_u32(&pv_done[(t - 1) % NS]), ((t - 1) / NS) & 1, kErrAttnConsumerWait);
-          tc_fence_after();
-          __syncwarp();
 #pragma unroll 1
-          for (int c0 = 0; c0 < OC; c0 += 16) {
+          for (int c0 = 0; c0 < D; c0 += 16) {
             uint32_t ov[16];
-            tmem_ld_cols<16>(lane_base + SM::kOCol + OC * part + c0, ov);
+            tmem_ld_cols<16>(o_col + c0, ov);
             tmem_ld_wait();
 #pragma unroll
             for (int k = 0; k < 16; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-            tmem_st_cols<16>(lane_base + SM::kOCol + OC * part + c0, ov);
+            tmem_st_cols<16>(o_col + c0, ov);
           }
           tmem_st_wait();
         }
@@ -364,37 +353,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           m_ref = m_new;
         }
         // p = 2^(s * scale_log2 - m), one fused multiply-add per score; masked keys give
-        // exp2(-inf) = 0 (and m = 0 while every key so far was masked)
-        const float c = prm.scale_log2;
+        // 2^-inf = 0 (and m = 0 while every key so far was masked)
         const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-        // P buffer t % 2 was last read by PV(t - 2)
-        if (t >= NS) mbar_wait(smem_u32(&pv_done[sb]), (t / NS - 1) & 1, kErrAttnConsumerWait);
-        uint32_t w[C / 2];
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t w[kTcHalf / 2];
+        float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < C / 2; ++e) {
-          const float p0 = fast_exp2(fmaf(x[2 * e], c, neg_m));
-          const float p1 = fast_exp2(fmaf(x[2 * e + 1], c, neg_m));
-          w[e] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < kTcHalf / 2; ++e) {
+          const float2 y = ffma2(make_float2(x[2 * e], x[2 * e + 1]), make_float2(c, c), make_float2(neg_m, neg_m));
+          float2 pe;
+          if ((e & 7) < kTcPolyPairs) {
+            pe = exp2_poly2(y);
+          } else {
+            pe.x = fast_exp2(y.x);
+            pe.y = fast_exp2(y.y);
+          }
+          w[e] = pack_bf16x2(pe.x, pe.y);
           // the denominator sums the fp32 values; the MMA multiplies their bf16 roundings
           // (round to nearest: the difference averages out far below the bf16 tolerance)
-          ls[e & 3] += p0 + p1;
+          if (e & 1)
+            ls1 = fadd2(ls1, pe);
+          else
+            ls0 = fadd2(ls0, pe);
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        __syncwarp();
-        tmem_st_cols<C / 2>(lane_base + SM::kPCol + sb * (kAttnKeys / 2) + (C / 2) * part, w);
+        ls0 = fadd2(ls0, ls1);
+        l += ls0.x + ls0.y;
+        // P_g was last read by PV_g(t - 1), complete like the rescale above
+        tmem_st_cols<32>(p_col, w);
         tmem_st_wait();
       }
       if (!tree) {
         const int valid = min(kAttnKeys, L - (t_begin + t) * kAttnKeys);
-        if (valid < kAttnKeys) {
+        const int lo = max(valid, grp * kTcHalf), hi = (grp + 1) * kTcHalf;
+        if (lo < hi) {
           // keys past L_b must not reach P V even if the padding holds non-finite values:
-          // zero those rows of this tile's V slot once it has landed
+          // zero this group's rows of them in the tile's V slot once it has landed
           const int s = t % SV;
           mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnConsumerWait);
           const uint32_t vb = v_stage(s);
-          for (int idx = tid; idx < (kAttnKeys - valid) * (D / 8); idx += kSoftThreads) {
-            const int j = valid + idx / (D / 8);
+          const int gtid = tid & 127;
+          for (int idx = gtid; idx < (hi - lo) * (D / 8); idx += 128) {
+            const int j = lo + idx / (D / 8);
             const int d = (idx % (D / 8)) * 8;
             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + attn_swz(j, d)), "r"(0));
           }
@@ -402,61 +400,67 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&p_full[sb]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&p_full[grp]));
     }
 
     // ------------------------------------------------------------ epilogue
-    // row denominator: this thread's columns plus the other parts'
-    if (live) {
-      float* lx = xch + 2 * kTcParts * kTcRows;
-      lx[part * kTcRows + r] = l;
-      quarter_sync();
-#pragma unroll
-      for (int o = 1; o < kTcParts; ++o) l += lx[((part + o) % kTcParts) * kTcRows + r];
-    }
+    // merge the two groups' partials: each publishes its (m, l) per row, then group g
+    // writes output columns [g D/2, (g + 1) D/2) from both accumulators
+    xch[(grp * 2 + 0) * kTcRows + r] = m_ref;
+    xch[(grp * 2 + 1) * kTcRows + r] = l;
+    asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+    const float m0 = xch[0 * kTcRows + r], l0 = xch[1 * kTcRows + r];
+    const float m1 = xch[2 * kTcRows + r], l1 = xch[3 * kTcRows + r];
+    const float mm = fmaxf(m0, m1);
+    const float f0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mm);
+    const float f1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mm);
+    const float lt = f0 * l0 + f1 * l1;
     if (T > 0) {
       mbar_wait(smem_u32(o_final), 0, kErrAttnConsumerWait);
       tc_fence_after();
     }
     const size_t prow_g = (static_cast<size_t>(b) * N + node) * prm.Hq + head;
     const bool single = prm.num_splits == 1;
-    const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+    const float inv = (lt > 0.f) ? 1.0f / lt : 0.f;
+    const uint32_t o0 = lane_base + SM::kOCol, o1 = lane_base + SM::kOCol + D;
     if (live) {
 #pragma unroll 1
-      for (int cc = 0; cc < OC; cc += 16) {
-        uint32_t ov[16];
-        __syncwarp();  // the TMEM load below is warp-wide
+      for (int cc = grp * (D / 2); cc < (grp + 1) * (D / 2); cc += 16) {
+        uint32_t a0[16], a1[16];
+        float ov[16];
+        __syncwarp();  // the TMEM loads below are warp-wide
         if (T > 0) {
-          tmem_ld_cols<16>(lane_base + SM::kOCol + OC * part + cc, ov);
+          tmem_ld_cols<16>(o0 + cc, a0);
+          tmem_ld_cols<16>(o1 + cc, a1);
           tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) ov[k] = f0 * __uint_as_float(a0[k]) + f1 * __uint_as_float(a1[k]);
         } else {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) ov[k] = 0u;
+          for (int k = 0; k < 16; ++k) ov[k] = 0.f;
         }
-        const int c0 = OC * part + cc;
         if (!rvalid) {
         } else if (single) {
-          uint4* dst = reinterpret_cast<uint4*>(prm.out + prow_g * D + c0);
+          uint4* dst = reinterpret_cast<uint4*>(prm.out + prow_g * D + cc);
 #pragma unroll
           for (int k = 0; k < 16; k += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ov[k + 2]) * inv, __uint_as_float(ov[k + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ov[k + 4]) * inv, __uint_as_float(ov[k + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ov[k + 6]) * inv, __uint_as_float(ov[k + 7]) * inv);
-            dst[k / 8] = w;
+            uint4 wv;
+            wv.x = pack_bf16x2(ov[k] * inv, ov[k + 1] * inv);
+            wv.y = pack_bf16x2(ov[k + 2] * inv, ov[k + 3] * inv);
+            wv.z = pack_bf16x2(ov[k + 4] * inv, ov[k + 5] * inv);
+            wv.w = pack_bf16x2(ov[k + 6] * inv, ov[k + 7] * inv);
+            dst[k / 8] = wv;
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(prm.part_acc + (prow_g * prm.num_splits + split) * D + c0);
+          float4* dst = reinterpret_cast<float4*>(prm.part_acc + (prow_g * prm.num_splits + split) * D + cc);
 #pragma unroll
-          for (int k = 0; k < 16; k += 4)
-            dst[k / 4] = make_float4(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1]),
-                                     __uint_as_float(ov[k + 2]), __uint_as_float(ov[k + 3]));
+          for (int k = 0; k < 16; k += 4) dst[k / 4] = make_float4(ov[k], ov[k + 1], ov[k + 2], ov[k + 3]);
         }
       }
     }
-    if (rvalid && !single && part == 0)
-      *reinterpret_cast<float2*>(prm.part_ml + (prow_g * prm.num_splits + split) * 2) = make_float2(m_ref, l);
+    if (rvalid && !single && grp == 0)
+      *reinterpret_cast<float2*>(prm.part_ml + (prow_g * prm.num_splits + split) * 2) = make_float2(mm, lt);
   }
 
   tc_fence_before();

@@ -411,4 +411,62 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Maximum of three values in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pairs: one sm_100 instruction does the work of two scalar ones (same pipe
+// throughput per value, half the issue slots).
+__device__ __forceinline__ uint64_t f2_bits(float2 v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+  return r;
+}
+__device__ __forceinline__ float2 bits_f2(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+
+// 2^y for a pair of values on the FMA and integer pipes instead of the SFU, to share the
+// exponentials of a softmax between the two.  Range reduction in the Cody-Waite manner:
+// y = j + f with j = round(y) (adding 1.5 * 2^23 leaves j in the low mantissa bits) and
+// |f| <= 1/2; 2^f from a cubic whose coefficients were fitted for the least maximum relative
+// error on [-1/2, 1/2] (1.0e-4, far below the bf16 rounding the result goes through); 2^j is
+// built directly in the exponent field.  y is clamped to >= -127, where that field is 0, so
+// -inf and everything below about -126.5 give exactly +0.  For y <= 128 only.
+__device__ __forceinline__ float2 exp2_poly2(float2 y) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  y.x = fmaxf(y.x, -127.0f);
+  y.y = fmaxf(y.y, -127.0f);
+  const float2 t = fadd2(y, make_float2(kShift, kShift));
+  const float2 j = fadd2(t, make_float2(-kShift, -kShift));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), y);
+  float2 q = ffma2(make_float2(0.0550089292f, 0.0550089292f), f, make_float2(0.242210954f, 0.242210954f));
+  q = ffma2(q, f, make_float2(0.693282902f, 0.693282902f));
+  q = ffma2(q, f, make_float2(1.0f, 1.0f));
+  // (j + 127) << 23: the low bits of t hold j + 2^22, whose shifted-out part vanishes
+  const float2 sc = make_float2(__uint_as_float((__float_as_uint(t.x) << 23) + 0x3F800000u),
+                                __uint_as_float((__float_as_uint(t.y) << 23) + 0x3F800000u));
+  return fmul2(q, sc);
+}
+
 }  // namespace eagle

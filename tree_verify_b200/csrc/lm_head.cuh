@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&acc_full[a]), 1);
-      mbar_init(smem_u32(&acc_empty[a]), 128);
+      mbar_init(smem_u32(&acc_empty[a]), 4);  // one arrival per epilogue warp
     }
     mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&acc_empty[a]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[a]));
     }
   }
   __syncwarp();

@@ -163,6 +163,29 @@ def test_lm_head_matches_oracle(cuda_lib, orc, case):
         assert err.max() <= 1e-5, f"max row error {err.max():.3e}"
 
 
+def test_lm_head_two_block_tiles_match_oracle(cuda_lib, orc):
+    """Enough vocabulary for the persistent kernel's two-block tiles (six or more tiles of
+    256 vocabulary rows per SM), with a ragged last tile whose second block lies past the
+    vocabulary: every logit written, sampled rows of both row chunks against the oracle."""
+    from tree_verify_b200.step import to_device
+    M, H, V = 300, 256, 113_500
+    rng = np.random.default_rng(2024)
+    hidden = _mk(rng, (M, H), "bf16")
+    w = wl.round_to_bf16_bits((rng.standard_normal((V, H)) / np.sqrt(H)).astype(np.float32))
+    shape = cuda_lib.make_shape(1, 1, 1, 1, 64, 1, H, V, "bf16")
+    shape.batch, shape.num_nodes = M, 1
+    logits = torch.full((M, V), float("nan"), dtype=torch.float32, device="cuda")
+    cuda_lib.lm_head_logits(shape, to_device(hidden, "bf16"), to_device(w, "bf16"), logits)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error(reset=True) == 0
+    got = logits.cpu().numpy()
+    assert np.isfinite(got).all()
+    rows = np.array([0, 1, 77, 149, 150, 151, 159, 160, 161, 230, 298, 299], dtype=np.int32)
+    ref = orc.lm_head(hidden, w, rows=rows)
+    err = row_rel_err(got[rows], ref)
+    assert err.max() <= 1e-5, f"max row error {err.max():.3e}"
+
+
 # ------------------------------------------------------------------ accept / resample
 
 def _accept_inputs(rng, B, N, V, T, max_depth=5, dup_draft=True):

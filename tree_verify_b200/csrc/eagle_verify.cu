@@ -237,7 +237,9 @@ bool ensure_attributes(int dev) {
     bool ok = true;
     ok &= cudaFuncSetAttribute(lm_head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) == cudaSuccess;
-    ok &= cudaFuncSetAttribute(lm_head_tc_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    ok &= cudaFuncSetAttribute(lm_head_tc_persist_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               227 * 1024) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(lm_head_tc_persist_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                227 * 1024) == cudaSuccess;
     ok &= cudaFuncSetAttribute(tree_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                TcSmem<64>::kAlloc) == cudaSuccess;
@@ -380,8 +382,10 @@ eagle_status_t run_attention(const eagle_shape_t* s, const void* q, const void* 
 }
 
 // Many tree rows (more than one chunk of 256): the persistent kernel, one CTA per SM, the
-// chunks of a vocabulary tile on neighbouring CTAs, the epilogue of one tile under the
-// MMAs of the next.
+// chunks of a vocabulary tile on neighbouring CTAs.  Tiles of two 128-row vocabulary blocks
+// (a third fewer shared-memory bytes per MMA; each tile's epilogue not overlapped) when
+// there are enough of them to keep the last round of tiles short (six per SM), else single
+// blocks with the epilogue of one tile under the MMAs of the next.
 eagle_status_t run_lm_head_persistent(const eagle_shape_t* s, const void* hidden, const void* w,
                                       float* logits, cudaStream_t st, const LmPlan& plan) {
   const int M = s->batch * s->num_nodes, V = s->vocab, H = s->hidden;
@@ -393,14 +397,19 @@ eagle_status_t run_lm_head_persistent(const eagle_shape_t* s, const void* hidden
   const cuuint32_t hbox[2] = {static_cast<cuuint32_t>(kLmBlockK), static_cast<cuuint32_t>(plan.bn)};
   if (!encode_bf16(&tw, w, 2, wd, stride, wbox) || !encode_bf16(&th, hidden, 2, hd, stride, hbox))
     return EAGLE_ERR_CUDA;
-  const int vtiles = (V + kLmBlockV - 1) / kLmBlockV;
+  const long wide_tiles = static_cast<long>((V + 2 * kLmBlockV - 1) / (2 * kLmBlockV)) * plan.chunks;
+  const int vb = wide_tiles >= 6L * kNumSMs ? 2 : 1;
+  const int vtiles = (V + vb * kLmBlockV - 1) / (vb * kLmBlockV);
   int stages = 2;
-  while (stages < 8 && lmp_smem_bytes(plan.bn, stages + 1) <= 220 * 1024) ++stages;
+  while (stages < 8 && lmp_smem_bytes(vb, plan.bn, stages + 1) <= 220 * 1024) ++stages;
   LmpParams prm{logits, M, V, H, plan.bn, plan.chunks, vtiles, stages};
-  const size_t smem = lmp_smem_bytes(plan.bn, stages);
+  const size_t smem = lmp_smem_bytes(vb, plan.bn, stages);
   const long tiles = static_cast<long>(vtiles) * plan.chunks;
   const int grid = static_cast<int>(tiles < kNumSMs ? tiles : kNumSMs);
-  lm_head_tc_persist_kernel<<<grid, kLmpThreads, smem, st>>>(tw, th, prm);
+  if (vb == 2)
+    lm_head_tc_persist_kernel<2><<<grid, kLmpThreads, smem, st>>>(tw, th, prm);
+  else
+    lm_head_tc_persist_kernel<1><<<grid, kLmpThreads, smem, st>>>(tw, th, prm);
   return launch_status();
 }
 

@@ -171,11 +171,16 @@ __global__ void __launch_bounds__(kLmThreads, 1)
 // For many tree rows (M > 256, where the GEMM is bound by the tensor cores rather than by
 // the weight stream): one CTA per SM walks a list of (vocabulary tile, row chunk) tiles,
 // row chunk fastest, so the CTAs working on the chunks of one vocabulary tile run side by
-// side and W is read from HBM about once.  Two TMEM accumulators (2 x 256 columns) let the
-// epilogue warps drain tile j while the MMAs of tile j + 1 run.  Warp roles: warp 0 lane 0
-// issues TMA (a W box and a hidden box per k block, one ring), warp 1 owns TMEM and lane 0
-// issues the MMAs, warps 2-5 drain TMEM (warp w reads TMEM lanes 32 * (w % 4) ..) and store
-// fp32 logits in coalesced 128-byte rows.
+// side and W is read from HBM about once.  Warp roles: warp 0 lane 0 issues TMA (W boxes and
+// a hidden box per k block, one ring), warp 1 owns TMEM and lane 0 issues the MMAs, warps 2-5
+// drain TMEM (warp w reads TMEM lanes 32 * (w % 4) ..) and store fp32 logits in coalesced
+// 128-byte rows.  Two tile shapes (kVB vocabulary blocks of 128 rows per tile):
+//   kVB = 1  two TMEM accumulators (2 x 256 columns): the epilogue drains tile j while the
+//            MMAs of tile j + 1 run;
+//   kVB = 2  one accumulator per block (the same 512 columns): every k block's hidden tile
+//            feeds two MMAs, so a tile moves a third fewer bytes through shared memory per
+//            MMA (the bound of this GEMM: TMA writes plus operand reads per stage), at the
+//            price of the MMAs waiting for each tile's epilogue.
 
 constexpr int kLmpThreads = 192;
 constexpr int kLmpAccCols = 256;  // columns per accumulator
@@ -185,24 +190,31 @@ struct LmpParams {
   int32_t M, V, H;
   int32_t bn;       // rows per chunk, multiple of 16, <= 256
   int32_t chunks;   // row chunks (ceil(M / bn))
-  int32_t vtiles;   // vocabulary tiles of 128
+  int32_t vtiles;   // vocabulary tiles of 128 * kVB
   int32_t stages;
 };
 
-__host__ __device__ inline size_t lmp_smem_bytes(int bn, int stages) {
-  return 1024 + static_cast<size_t>(stages) * lm_stage_bytes(bn) + (2 * stages + 5) * 8 + 16;
+__host__ __device__ inline uint32_t lmp_stage_bytes(int vb, int bn) {
+  return static_cast<uint32_t>(vb * kLmBlockV * kLmBlockK * 2 + bn * kLmBlockK * 2);
+}
+__host__ __device__ inline size_t lmp_smem_bytes(int vb, int bn, int stages) {
+  return 1024 + static_cast<size_t>(stages) * lmp_stage_bytes(vb, bn) + (2 * stages + 5) * 8 + 16;
 }
 
+template <int kVB>
 __global__ void __launch_bounds__(kLmpThreads, 1)
     lm_head_tc_persist_kernel(const __grid_constant__ CUtensorMap tm_w,
                               const __grid_constant__ CUtensorMap tm_h, const LmpParams prm) {
+  static_assert(kVB == 1 || kVB == 2, "one or two vocabulary blocks per tile");
+  constexpr int NA = kVB == 1 ? 2 : 1;  // accumulator sets in flight
+  constexpr uint32_t kWBox = kLmBlockV * kLmBlockK * 2;
   extern __shared__ uint8_t lmp_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lmp_smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int S = prm.stages;
   const int bn = prm.bn;
-  uint8_t* a_tiles = smem;                                    // S x 16 KB
-  uint8_t* b_tiles = smem + S * kLmBlockV * kLmBlockK * 2;    // S x bn*128 B
+  uint8_t* a_tiles = smem;                                    // S x kVB x 16 KB
+  uint8_t* b_tiles = smem + S * kVB * kWBox;                  // S x bn*128 B
   uint64_t* bars = reinterpret_cast<uint64_t*>(b_tiles + S * bn * kLmBlockK * 2);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
@@ -245,11 +257,11 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
-      const uint32_t bytes = lm_stage_bytes(bn);
+      const uint32_t bytes = lmp_stage_bytes(kVB, bn);
       const uint64_t pol_h = l2_policy_evict_last();  // every tile re-reads hidden
       int it = 0, issued = 0;
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-        const int c = tile % prm.chunks, v0 = (tile / prm.chunks) * kLmBlockV;
+        const int c = tile % prm.chunks, v0 = (tile / prm.chunks) * (kVB * kLmBlockV);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S, n = it / S;
           if (n > 0 && !mbar_wait(smem_u32(&empty[s]), (n - 1) & 1, kErrLmProducerWait)) {
@@ -258,7 +270,10 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
           }
           const uint32_t fb = smem_u32(&full[s]);
           mbar_arrive_expect_tx(fb, bytes);
-          tma_load_2d(smem_u32(a_tiles + s * kLmBlockV * kLmBlockK * 2), &tm_w, fb, kb * kLmBlockK, v0);
+#pragma unroll
+          for (int vb = 0; vb < kVB; ++vb)
+            tma_load_2d(smem_u32(a_tiles + (s * kVB + vb) * kWBox), &tm_w, fb, kb * kLmBlockK,
+                        v0 + vb * kLmBlockV);
           tma_load_2d_hint(smem_u32(b_tiles + s * bn * kLmBlockK * 2), &tm_h, fb, kb * kLmBlockK, c * bn,
                            pol_h);
           issued = it + 1;
@@ -274,12 +289,13 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(kLmBlockV, bn);
       int it = 0, j = 0;
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, ++j) {
-        const int a = j & 1;
-        if (j >= 2 && !mbar_wait(smem_u32(&acc_empty[a]), ((j - 2) >> 1) & 1, kErrLmMmaWait)) {
+        const int a = j % NA;
+        if (j >= NA && !mbar_wait(smem_u32(&acc_empty[a]), (j / NA - 1) & 1, kErrLmMmaWait)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
+        // accumulator of block vb: set a (kVB = 1) or block vb (kVB = 2), 256 columns each
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(a * kLmpAccCols);
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -289,11 +305,15 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t a_desc = smem_desc_k_sw128(smem_u32(a_tiles + s * kLmBlockV * kLmBlockK * 2));
           const uint64_t b_desc = smem_desc_k_sw128(smem_u32(b_tiles + s * bn * kLmBlockK * 2));
 #pragma unroll
           for (int k = 0; k < kLmBlockK / 16; ++k)
-            tc_mma_f16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int vb = 0; vb < kVB; ++vb) {
+              const uint64_t a_desc = smem_desc_k_sw128(smem_u32(a_tiles + (s * kVB + vb) * kWBox));
+              tc_mma_f16(d_tmem + static_cast<uint32_t>(vb * kLmpAccCols), a_desc + 2 * k, b_desc + 2 * k, idesc,
+                         (kb | k) != 0 ? 1u : 0u);
+            }
           tc_commit(smem_u32(&empty[s]));
         }
         if (!ok) {
@@ -310,27 +330,30 @@ __global__ void __launch_bounds__(kLmpThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int j = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++j) {
-      const int a = j & 1;
-      if (!mbar_wait(smem_u32(&acc_full[a]), (j >> 1) & 1, kErrLmEpilogueWait)) {
+      const int a = j % NA;
+      if (!mbar_wait(smem_u32(&acc_full[a]), (j / NA) & 1, kErrLmEpilogueWait)) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const int c = tile % prm.chunks, v0 = (tile / prm.chunks) * kLmBlockV;
-      const int v = v0 + q * 32 + lane;
+      const int c = tile % prm.chunks, v0 = (tile / prm.chunks) * (kVB * kLmBlockV);
       const int r0 = c * bn;
-      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(a * kLmpAccCols);
       float* out = prm.logits;
-      for (int c0 = 0; c0 < bn; c0 += 16) {
-        uint32_t r[16];
-        __syncwarp();  // the TMEM load below is warp-wide
-        tmem_ld_32x32b_x16(lane_base + c0, r);
-        tmem_ld_wait();
-        if (v < prm.V) {
+      for (int vb = 0; vb < kVB; ++vb) {
+        const int v = v0 + vb * kLmBlockV + q * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>((a + vb) * kLmpAccCols);
+        for (int c0 = 0; c0 < bn; c0 += 16) {
+          uint32_t r[16];
+          __syncwarp();  // the TMEM load below is warp-wide
+          tmem_ld_32x32b_x16(lane_base + c0, r);
+          tmem_ld_wait();
+          if (v < prm.V) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int row = r0 + c0 + e;
-            if (row < prm.M) out[static_cast<size_t>(row) * prm.V + v] = __uint_as_float(r[e]);
+            for (int e = 0; e < 16; ++e) {
+              const int row = r0 + c0 + e;
+              if (row < prm.M) out[static_cast<size_t>(row) * prm.V + v] = __uint_as_float(r[e]);
+            }
           }
         }
       }

@@ -139,7 +139,8 @@ eagle_status_t eagle_lm_head_logits(const eagle_shape_t *shape, const void *hidd
  * sample is the exponential race argmin_v -ln u(b, cur, v, 1) / p_v, lowest v on ties.
  *   logits          [B,N,V] float32 (the output of eagle_lm_head_logits)
  *   draft_probs     [B,N,V] float32; row c = the distribution node c was drafted from
- *                   (row 0 unused); read only for tested candidates
+ *                   (row 0 unused); at T > 0 entry (c, tokens[c]) of every drafted node
+ *                   and the whole row only of tested candidates are read
  *   tokens          [B,N] int32; tokens[b,0] is the committed root token (unused)
  *   parents         [B,N] int32
  *   temperature     >= 0

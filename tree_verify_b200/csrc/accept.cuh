@@ -108,8 +108,8 @@ struct AccShared {
   int32_t child_start[65];
   int32_t child_list[64];
   int32_t acc_nodes[64];
-  float qx[64];                        // p_hat_c(t_c) of the current node's children
-  float ux[64];                        // accept-test uniforms
+  float qx[64];                        // p_hat_c(t_c) of every drafted node c (T > 0)
+  float ux[64];                        // node c's accept-test uniform (T > 0)
 };
 
 // Butterfly over lanes `offs..1` that moves only the first NC components (the ones the
@@ -337,6 +337,13 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     fence_mbar_init();
   }
   ok = __syncthreads_and(ok);
+  if (ok && T > 0.f && tid >= 1 && tid < N) {
+    // what the accept test of node tid needs besides the target row: the draft probability
+    // of its token in the row it was drafted from, and its uniform; loaded once here, before
+    // the LM head has finished, rather than on the walk's path
+    sh.qx[tid] = prm.draft[(seq + tid) * V + sh.tok[tid]];
+    sh.ux[tid] = uniform_at(prm.seed, prm.offset, b, tid, 0, 0);
+  }
   if (ok && tid <= N) {
     // start of node u's children list = number of drafted nodes whose parent is < u
     int start = 0;
@@ -394,7 +401,8 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     done_sent = true;
   };
 
-  // draft side of a node: candidate rows, p_hat_c(t_c) and the accept uniforms
+  // draft side of a node: the candidates' draft rows (their p_hat_c(t_c) and uniforms were
+  // loaded for every node at set-up)
   auto issue_draft = [&](int node) {
     const int c_begin = sh.child_start[node];
     const int kids = sh.child_start[node + 1] - c_begin;
@@ -407,11 +415,6 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
       __syncthreads();
     }
     for (int j = 0; j < pre; ++j) fetch_q(j, sh.child_list[c_begin + j]);
-    if (tid < kids) {
-      const int c = sh.child_list[c_begin + tid];
-      sh.qx[tid] = prm.draft[(seq + c) * V + sh.tok[c]];
-      sh.ux[tid] = uniform_at(prm.seed, prm.offset, b, c, 0, 0);
-    }
   };
   // ebuf holds the race keys of node `ekey`: the root's, computed now (the walk most often
   // ends there), later those of each visited node, computed while its first reduction
@@ -440,7 +443,7 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     fetch_slice<kBulk>(rowbuf, row + v_lo, n_loc, &sh.row_bar);
     if (depth > 0 && T > 0.f) issue_draft(cur);
     failed |= !wait_slice<kBulk>(&sh.row_bar, row_phase, n_loc);
-    __syncthreads();  // qx / ux visible
+    __syncthreads();  // the row slice is in shared memory for every thread
 
     if (T == 0.f) {
       // greedy: argmax of the target logits, lowest index on ties
@@ -518,8 +521,8 @@ __global__ void __launch_bounds__(kAccThreads, 1) tree_accept_kernel(const AccPa
     for (int j = 0; j < kids; ++j) {
       const int c = sh.child_list[c_begin + j];
       const float px = px_next;
-      const float qx = sh.qx[j];
-      if (qx == 0.f || sh.ux[j] < px / qx) {
+      const float qx = sh.qx[c];
+      if (qx == 0.f || sh.ux[c] < px / qx) {
         j_acc = j;
         break;
       }

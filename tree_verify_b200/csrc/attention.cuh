@@ -162,11 +162,21 @@ __global__ void __launch_bounds__(128)
     float s = -INFINITY;
     if (j < nk) {
       const float* kr = key_row(j, kp, kt);
+      // the whole key row is loaded before the dot product starts (one round trip)
+      float kv[D];
+#pragma unroll
+      for (int d = 0; d < D; d += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kr + d);
+        kv[d] = k4.x;
+        kv[d + 1] = k4.y;
+        kv[d + 2] = k4.z;
+        kv[d + 3] = k4.w;
+      }
       float d0 = 0.f, d1 = 0.f;
-#pragma unroll 8
+#pragma unroll
       for (int d = 0; d < D; d += 2) {
-        d0 = fmaf(q_s[wid][d], kr[d], d0);
-        d1 = fmaf(q_s[wid][d + 1], kr[d + 1], d1);
+        d0 = fmaf(q_s[wid][d], kv[d], d0);
+        d1 = fmaf(q_s[wid][d + 1], kv[d + 1], d1);
       }
       s = (d0 + d1) * scale;
     }
@@ -183,11 +193,23 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int e = 0; e < kPer; ++e) acc[e] *= corr;
     const int cnt = min(32, nk - c);
-    for (int t = 0; t < cnt; ++t) {
-      const float pt = __shfl_sync(0xffffffffu, p, t);
-      const float* vr = key_row(c + t, vp, vt);
+    // eight keys' V loads in flight before their products are added (in key order)
+    for (int t0 = 0; t0 < cnt; t0 += 8) {
+      float vv[8][kPer];
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) acc[e] = fmaf(pt, vr[lane + 32 * e], acc[e]);
+      for (int t = 0; t < 8; ++t) {
+        const float* vr = key_row(min(c + t0 + t, nk - 1), vp, vt);
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) vv[t][e] = vr[lane + 32 * e];
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float pt = __shfl_sync(0xffffffffu, p, t0 + t < 32 ? t0 + t : 31);
+        if (t0 + t < cnt) {
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) acc[e] = fmaf(pt, vv[t][e], acc[e]);
+        }
+      }
     }
     m = mn;
   }

@@ -392,15 +392,33 @@ __global__ void __launch_bounds__(256)
   const int r0 = blockIdx.y * kLmF32TileR;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int k0 = 0; k0 < H; k0 += kLmF32TileK) {
-    for (int idx = threadIdx.x; idx < kLmF32TileV * kLmF32TileK; idx += blockDim.x) {
+    // every load of the tile is issued before any is stored, so a tile costs one memory
+    // round trip (a load-store loop would wait for each load in turn)
+    constexpr int kWPer = kLmF32TileV * kLmF32TileK / 256, kHPer = kLmF32TileR * kLmF32TileK / 256;
+    float wr[kWPer], hr[kHPer];
+#pragma unroll
+    for (int e = 0; e < kWPer; ++e) {
+      const int idx = threadIdx.x + e * 256;
       const int vv = idx / kLmF32TileK, kk = idx % kLmF32TileK;
       const int gv = v0 + vv, gk = k0 + kk;
-      ws[vv][kk] = (gv < V && gk < H) ? w[static_cast<size_t>(gv) * H + gk] : 0.f;
+      wr[e] = (gv < V && gk < H) ? w[static_cast<size_t>(gv) * H + gk] : 0.f;
     }
-    for (int idx = threadIdx.x; idx < kLmF32TileR * kLmF32TileK; idx += blockDim.x) {
+#pragma unroll
+    for (int e = 0; e < kHPer; ++e) {
+      const int idx = threadIdx.x + e * 256;
       const int rr = idx / kLmF32TileK, kk = idx % kLmF32TileK;
       const int gr = r0 + rr, gk = k0 + kk;
-      hs[rr][kk] = (gr < M && gk < H) ? hidden[static_cast<size_t>(gr) * H + gk] : 0.f;
+      hr[e] = (gr < M && gk < H) ? hidden[static_cast<size_t>(gr) * H + gk] : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < kWPer; ++e) {
+      const int idx = threadIdx.x + e * 256;
+      ws[idx / kLmF32TileK][idx % kLmF32TileK] = wr[e];
+    }
+#pragma unroll
+    for (int e = 0; e < kHPer; ++e) {
+      const int idx = threadIdx.x + e * 256;
+      hs[idx / kLmF32TileK][idx % kLmF32TileK] = hr[e];
     }
     __syncthreads();
 #pragma unroll 8

@@ -8,31 +8,36 @@
 // every prefix K/V tile is read from HBM once.
 //
 // Keys arrive in tiles of 128 (one TMA box per 64 columns of D).  Each tile is split
-// between two softmax groups: group 0 takes keys 0-63 of every tile, group 1 keys 64-127.
-// A group keeps its own running maximum, denominator and output accumulator O_g, so the
-// two groups never wait for each other: while one exponentiates (SFU and FMA pipes), the
-// other loads scores and takes maxima, and the tensor core runs the other group's MMAs.
-// The two partial results are merged by log-sum-exp at the end.
+// between two softmax groups: group 0 takes keys 0-63 of every tile, group 1 keys 64-127,
+// one thread per query row in each.  The two threads of a row swap their halves' maxima
+// through shared memory once per tile, so both take the same running maximum, and their
+// P values feed one output accumulator O: per tile the tensor core runs two MMA chains
+// (S and PV), and a switch between chains with different accumulators costs it a pipeline
+// drain of a few hundred clocks.
 //
-//   warps 0-3 / 4-7   softmax groups 0 / 1: one thread per query row (TMEM lane = row,
-//                     warp w serves lane quarter w % 4): tcgen05.ld of the group's 64
-//                     scores, mask (prefix length, or the ancestor bitmask on the tree
-//                     tile), row maximum, P = 2^(s * c - m), tcgen05.st of P (bf16 pairs);
+//   warps 0-3 / 4-7   softmax groups 0 / 1 (TMEM lane = row, warp w serves lane quarter
+//                     w % 4): tcgen05.ld of the group's 64 scores, mask (prefix length, or
+//                     the ancestor bitmask on the tree tile), the half's maximum, the swap,
+//                     P = 2^(s * c - m), tcgen05.st of P (bf16 pairs);
 //   warp 8 lane 0     TMA: the Q tile once (a 3-D box over [B*N, Hq, D]), then the K tiles;
-//   warp 8 lane 1     TMA: the V tiles (their own ring, so a K slot refills as soon as both
+//   warp 8 lane 1     TMA: the V tiles (their own ring, so a K slot refills as soon as the
 //                     S MMAs have read it, ahead of its V slot);
-//   warp 9 lane 0     tcgen05.mma: S_g = Q K_g^T (M 128, N 64, K = D) and O_g += P_g V_g
-//                     (M 128, N = D, K 64; P read from TMEM, V an MN-major operand straight
-//                     from its TMA tile);
+//   warp 9 lane 0     tcgen05.mma: S = Q K^T (M 128, N 128, K = D) and O += P V (M 128,
+//                     N = D, K 128; P read from TMEM, V an MN-major operand straight from
+//                     its TMA tile), in the order PV(t), S(t + 2);
 //   warps 10-11       no role (a 384-thread block caps registers at 168, which three warps
 //                     per SM sub-partition can hold).
-// TMEM: S_0 S_1 (64 columns each), P_0 P_1 (32), O_0 O_1 (D each).  O_g is rescaled lazily,
-// only when the group's row maximum grows by more than 2^8 over the reference its P values
-// were taken against.  A commit on s_full_g(t) covers every earlier MMA, PV_g(t-1) included,
-// so a group that sees S_g(t) may overwrite P_g and rescale O_g.  The last split also runs
-// the tree tile: its K/V rows come by TMA from a 4-D view of the tree K/V ([B][N][Hkv][D],
-// rows past N zero-filled).  Splits write (m, l, acc) partials for the log-sum-exp merge; a
-// single split normalises and writes the output.
+// TMEM: two S buffers of 128 columns, then O (D columns).  S(t) goes to buffer t % 2, so
+// the tensor core computes S(t + 1) while the groups work on tile t; the bf16 P of each
+// half is written over the first 32 columns of that half of S(t).  The MMAs of one CTA run
+// in issue order, so S(t + 2), issued after PV(t), overwrites P(t) only once PV(t) has read
+// it.  The groups wait for PV(t - 1) (pv_done) before they rescale O, and before they
+// announce P(t), so they never run two barrier phases ahead of the MMA issuer.  O is
+// rescaled lazily (each group its half of the columns), only when the row maximum grows by
+// more than 2^8 over the reference the P values were taken against.  The last split also
+// runs the tree tile: its K/V rows come by TMA from a 4-D view of the tree K/V
+// ([B][N][Hkv][D], rows past N zero-filled).  Splits write (m, l, acc) partials for the
+// log-sum-exp merge; a single split normalises and writes the output.
 #pragma once
 
 #include "attention.cuh"
@@ -63,18 +68,22 @@ struct TcSmem {
   static constexpr int kVOff = kKOff + kKStages * kTile;
   static constexpr int kAncOff = kVOff + kVStages * kTile;
   static constexpr int kParOff = kAncOff + 64 * 8;
-  // the groups' (m, l) per row for the final merge: [group][2][row]
+  // the halves' maxima per row and tile parity, [parity][group][row]; then the groups'
+  // denominators per row for the epilogue, [group][row]
   static constexpr int kXchOff = kParOff + 64 * 4;
-  static constexpr int kBarOff = kXchOff + 2 * 2 * kTcRows * 4;
-  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2], p_full[2], o_final
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 1;
+  static constexpr int kLOff = kXchOff + 2 * 2 * kTcRows * 4;
+  static constexpr int kBarOff = kLOff + 2 * kTcRows * 4;
+  // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[buffer], p_full,
+  // pv_done, o_final
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 1 + 1 + 1;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  // TMEM columns
-  static constexpr uint32_t kSCol = 0;                  // S_g at kSCol + 64 g
-  static constexpr uint32_t kPCol = 2 * kTcHalf;        // P_g at kPCol + 32 g
-  static constexpr uint32_t kOCol = 256;                // O_g at kOCol + D g
+  // TMEM columns: S(t) in buffer u = t % 2 at kSCol + kAttnKeys u (keys in column order;
+  // the P of group g over the kTcHalf / 2 columns from kTcHalf g), O at kOCol
+  static constexpr uint32_t kSCol = 0;
+  static constexpr uint32_t kOCol = 2 * kAttnKeys;
   static constexpr uint32_t kTmemCols = 512;
+  static_assert(kOCol + D <= kTmemCols, "TMEM columns");
 };
 
 struct TcAttnParams {
@@ -98,15 +107,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* anc = reinterpret_cast<uint64_t*>(smem + SM::kAncOff);
   int32_t* par_s = reinterpret_cast<int32_t*>(smem + SM::kParOff);
   float* xch = reinterpret_cast<float*>(smem + SM::kXchOff);
+  float* l_s = reinterpret_cast<float*>(smem + SM::kLOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBarOff);
   uint64_t* q_full = bars;
   uint64_t* k_full = q_full + 1;
   uint64_t* k_empty = k_full + SK;
   uint64_t* v_full = k_empty + SK;
   uint64_t* v_empty = v_full + SV;
-  uint64_t* s_full = v_empty + SV;  // [group]
-  uint64_t* p_full = s_full + 2;    // [group]
-  uint64_t* o_final = p_full + 2;
+  uint64_t* s_full = v_empty + SV;  // [buffer]
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint64_t* o_final = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -139,10 +150,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
     }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(smem_u32(&s_full[g]), 1);
-      mbar_init(smem_u32(&p_full[g]), 4);  // one arrival per warp of the group
-    }
+    for (int u = 0; u < 2; ++u) mbar_init(smem_u32(&s_full[u]), 1);
+    mbar_init(smem_u32(p_full), kTcSoftmaxWarps);  // one arrival per softmax warp
+    mbar_init(smem_u32(pv_done), 1);
     mbar_init(smem_u32(o_final), 1);
     fence_mbar_init();
   }
@@ -201,18 +211,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == kTcMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kTcRows, kTcHalf);
+      const uint32_t idesc_s = idesc_bf16_f32(kTcRows, kAttnKeys);
       const uint32_t idesc_o = idesc_bf16_f32_bmn(kTcRows, D);
       bool ok = mbar_wait(smem_u32(q_full), 0, kErrAttnMmaWait);
-      // S_g(t) = Q K^T over keys [64 g, 64 g + 64) of tile t.  Buffer S_g was last read by
-      // the group's softmax of tile t - 1, which finished before its p_full arrival, and
-      // that was waited for before PV_g(t - 1) was issued.
-      auto issue_s = [&](int t, int g) {
+      // S(t) = Q K^T over the 128 keys of tile t, one M 128 x N 128 chain into buffer t % 2.
+      // That buffer last held S(t - 2) and P(t - 2): both groups arrived on p_full before
+      // PV(t - 2) was issued, and PV(t - 2) was issued before this chain.
+      auto issue_s = [&](int t) {
         const int s = t % SK;
-        if (g == 0) ok = ok && mbar_wait(smem_u32(&k_full[s]), (t / SK) & 1, kErrAttnMmaWait);
+        ok = ok && mbar_wait(smem_u32(&k_full[s]), (t / SK) & 1, kErrAttnMmaWait);
         tc_fence_after();
-        const uint32_t kb = k_stage(s) + static_cast<uint32_t>(g * kTcHalf * 128);
-        const uint32_t d_tmem = tmem + SM::kSCol + static_cast<uint32_t>(g * kTcHalf);
+        const uint32_t kb = k_stage(s);
+        const uint32_t d_tmem = tmem + SM::kSCol + static_cast<uint32_t>((t & 1) * kAttnKeys);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int h = kk >> 2, k4 = kk & 3;
@@ -220,35 +230,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t bdesc = smem_desc_k_sw128(kb + h * kAttnKeys * 128) + 2 * k4;
           if (ok) tc_mma_f16(d_tmem, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[g]));
-        if (g == 1) tc_commit(smem_u32(&k_empty[s]));  // both halves of the K slot are read
+        tc_commit(smem_u32(&s_full[t & 1]));
+        tc_commit(smem_u32(&k_empty[s]));
       };
-      // O_g += P_g V over the group's 64 keys: 4 MMAs of 16 keys (8 TMEM columns of P, two
-      // 8-key groups of 1024 B of V; the second 64-column group of V is the next TMA box)
-      auto issue_pv = [&](int t, int g) {
+      // O += P V over the tile's 128 keys: 8 MMAs of 16 keys (8 TMEM columns of P from the
+      // half that holds them, two 8-key groups of 1024 B of V; the second 64-column group
+      // of V is the next TMA box)
+      auto issue_pv = [&](int t) {
         const int s = t % SV;
-        ok = ok && mbar_wait(smem_u32(&p_full[g]), t & 1, kErrAttnMmaWait);
-        if (g == 0) ok = ok && mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnMmaWait);
+        ok = ok && mbar_wait(smem_u32(p_full), t & 1, kErrAttnMmaWait);
+        ok = ok && mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnMmaWait);
         tc_fence_after();
-        const uint32_t vb = v_stage(s) + static_cast<uint32_t>(g * kTcHalf * 128);
-        const uint32_t pa = tmem + SM::kPCol + static_cast<uint32_t>(g * (kTcHalf / 2));
-        const uint32_t o_tmem = tmem + SM::kOCol + static_cast<uint32_t>(g * D);
+        const uint32_t vb = v_stage(s);
+        const uint32_t pa = tmem + SM::kSCol + static_cast<uint32_t>((t & 1) * kAttnKeys);
+        const uint32_t o_tmem = tmem + SM::kOCol;
 #pragma unroll
-        for (int kk = 0; kk < kTcHalf / 16; ++kk) {
+        for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
+          const uint32_t a_col = static_cast<uint32_t>((kk >> 2) * kTcHalf + 8 * (kk & 3));
           const uint64_t bdesc = smem_desc_mn_sw128(vb + kk * 2048, kAttnKeys * 128, 1024);
-          if (ok) tc_mma_f16_ts(o_tmem, pa + 8 * kk, bdesc, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
+          if (ok) tc_mma_f16_ts(o_tmem, pa + a_col, bdesc, idesc_o, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        if (g == 1) tc_commit(smem_u32(&v_empty[s]));
+        tc_commit(smem_u32(pv_done));
+        tc_commit(smem_u32(&v_empty[s]));
       };
-      if (T > 0) {
-        issue_s(0, 0);
-        issue_s(0, 1);
-      }
+      for (int t = 0; t < T && t < 2; ++t) issue_s(t);
       for (int t = 0; t < T; ++t) {
-        issue_pv(t, 0);
-        if (t + 1 < T) issue_s(t + 1, 0);
-        issue_pv(t, 1);
-        if (t + 1 < T) issue_s(t + 1, 1);
+        issue_pv(t);
+        if (t + 2 < T) issue_s(t + 2);
       }
       tc_commit(smem_u32(o_final));
     }
@@ -284,15 +292,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // the tree keys are nodes 0..N-1 <= 63: all in group 0's half of the tree tile
     const uint64_t tree_bits = (last && rvalid && grp == 0) ? anc[node] : 0ull;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t s_col = lane_base + SM::kSCol + static_cast<uint32_t>(grp * kTcHalf);
-    const uint32_t p_col = lane_base + SM::kPCol + static_cast<uint32_t>(grp * (kTcHalf / 2));
-    const uint32_t o_col = lane_base + SM::kOCol + static_cast<uint32_t>(grp * D);
+    // the half of O's columns this group rescales and writes out
+    const uint32_t o_col = lane_base + SM::kOCol + static_cast<uint32_t>(grp * (D / 2));
     const float c = prm.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     for (int t = 0; t < T; ++t) {
       const bool tree = t >= nt;
-      mbar_wait(smem_u32(&s_full[grp]), t & 1, kErrAttnConsumerWait);
+      mbar_wait(smem_u32(&s_full[t & 1]), (t >> 1) & 1, kErrAttnConsumerWait);
       tc_fence_after();
+      // this group's half of S(t), and its P(t) over the half's first 32 columns
+      const uint32_t s_col = lane_base + SM::kSCol + static_cast<uint32_t>((t & 1) * kAttnKeys + grp * kTcHalf);
+      float tmax_half = -INFINITY;
+      float x[kTcHalf];
       if (live) {
         uint32_t sa[32], sb[32];
         __syncwarp();  // the TMEM loads below are warp-wide
@@ -307,7 +318,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!rvalid) vis = 0ull;
         // raw scores; masked ones (past L_b, outside the ancestor set, padding rows) become
         // -inf, which also drops any non-finite value the padding holds
-        float x[kTcHalf];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           x[j] = __uint_as_float(sa[j]);
@@ -327,27 +337,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int j = 0; j < 7; ++j) n3[j] = fmax3f(m3[3 * j], m3[3 * j + 1], m3[3 * j + 2]);
         n3[7] = m3[21];
         // in scaled log2 units (the scale is positive, so the maximum commutes with it)
-        const float tmax =
+        tmax_half =
             fmax3f(fmax3f(n3[0], n3[1], n3[2]), fmax3f(n3[3], n3[4], n3[5]), fmaxf(n3[6], n3[7])) * c;
+      }
+      // swap the halves' maxima: both threads of a row take the same maximum, so their P
+      // values share one reference and one accumulator.  The slot of tile t is written again
+      // at tile t + 2, after the other group has passed the swap of tile t + 1.
+      float* xm = xch + (t & 1) * 2 * kTcRows;
+      xm[grp * kTcRows + r] = tmax_half;
+      asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
+      const float tmax = fmaxf(tmax_half, xm[(grp ^ 1) * kTcRows + r]);
+      if (live) {
         const float m_new = fmaxf(m_ref, tmax);
         const bool rebase =
             m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kTcRescaleThreshold);
-        const bool scale_o = rebase && m_ref != -INFINITY;  // O_g holds P V taken against m_ref
+        const bool scale_o = rebase && m_ref != -INFINITY;  // O holds P V taken against m_ref
         const float f = scale_o ? fast_exp2(m_ref - m_new) : 1.0f;
-        // TMEM loads/stores are warp-wide: the warp rescales if any of its rows must.
-        // PV_g(t - 1) is complete: s_full_g(t) was committed after it.
-        if (__any_sync(0xffffffffu, scale_o)) {
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t ov[16];
-            tmem_ld_cols<16>(o_col + c0, ov);
-            tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 16; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-            tmem_st_cols<16>(o_col + c0, ov);
-          }
-          tmem_st_wait();
-        }
         if (rebase) {
           l *= f;
           m_ref = m_new;
@@ -377,8 +382,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         ls0 = fadd2(ls0, ls1);
         l += ls0.x + ls0.y;
-        // P_g was last read by PV_g(t - 1), complete like the rescale above
-        tmem_st_cols<32>(p_col, w);
+        // every score of this half of S(t) is in registers: its P goes over them
+        tmem_st_cols<32>(s_col, w);
+        // O holds P V taken against the old reference: rescale this group's half of its
+        // columns once PV(t - 1) has landed.  TMEM loads/stores are warp-wide: the warp
+        // rescales if any of its rows must (the other group's warp on the same rows decides
+        // the same).
+        if (__any_sync(0xffffffffu, scale_o)) {
+          if (t > 0) mbar_wait(smem_u32(pv_done), (t - 1) & 1, kErrAttnConsumerWait);
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < D / 2; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld_cols<16>(o_col + c0, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+            tmem_st_cols<16>(o_col + c0, ov);
+          }
+        }
         tmem_st_wait();
       }
       if (!tree) {
@@ -399,23 +421,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
       }
+      // PV(t - 1) issued means the issuer has taken p_full phase t - 1: arriving for phase t
+      // cannot complete two phases ahead of its wait
+      if (t > 0) mbar_wait(smem_u32(pv_done), (t - 1) & 1, kErrAttnConsumerWait);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&p_full[grp]));
+      if (lane == 0) mbar_arrive(smem_u32(p_full));
     }
 
     // ------------------------------------------------------------ epilogue
-    // merge the two groups' partials: each publishes its (m, l) per row, then group g
-    // writes output columns [g D/2, (g + 1) D/2) from both accumulators
-    xch[(grp * 2 + 0) * kTcRows + r] = m_ref;
-    xch[(grp * 2 + 1) * kTcRows + r] = l;
+    // both groups hold the same m_ref; the row's denominator is the sum of the halves'
+    l_s[grp * kTcRows + r] = l;
     asm volatile("bar.sync 1, %0;" ::"r"(kSoftThreads) : "memory");
-    const float m0 = xch[0 * kTcRows + r], l0 = xch[1 * kTcRows + r];
-    const float m1 = xch[2 * kTcRows + r], l1 = xch[3 * kTcRows + r];
-    const float mm = fmaxf(m0, m1);
-    const float f0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mm);
-    const float f1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mm);
-    const float lt = f0 * l0 + f1 * l1;
+    const float mm = m_ref;
+    const float lt = l_s[r] + l_s[kTcRows + r];
     if (T > 0) {
       mbar_wait(smem_u32(o_final), 0, kErrAttnConsumerWait);
       tc_fence_after();
@@ -423,19 +442,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const size_t prow_g = (static_cast<size_t>(b) * N + node) * prm.Hq + head;
     const bool single = prm.num_splits == 1;
     const float inv = (lt > 0.f) ? 1.0f / lt : 0.f;
-    const uint32_t o0 = lane_base + SM::kOCol, o1 = lane_base + SM::kOCol + D;
     if (live) {
 #pragma unroll 1
       for (int cc = grp * (D / 2); cc < (grp + 1) * (D / 2); cc += 16) {
-        uint32_t a0[16], a1[16];
+        uint32_t a0[16];
         float ov[16];
         __syncwarp();  // the TMEM loads below are warp-wide
         if (T > 0) {
-          tmem_ld_cols<16>(o0 + cc, a0);
-          tmem_ld_cols<16>(o1 + cc, a1);
+          tmem_ld_cols<16>(lane_base + SM::kOCol + cc, a0);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 16; ++k) ov[k] = f0 * __uint_as_float(a0[k]) + f1 * __uint_as_float(a1[k]);
+          for (int k = 0; k < 16; ++k) ov[k] = __uint_as_float(a0[k]);
         } else {
 #pragma unroll
           for (int k = 0; k < 16; ++k) ov[k] = 0.f;

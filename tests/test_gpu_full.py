@@ -125,3 +125,42 @@ def test_verify_step_stages_equal_fused_call(cuda_lib):
     assert cuda_lib.device_error(reset=True) == 0
     for name in ("out", "logits", "accepted_nodes", "accept_len", "next_token"):
         assert torch.equal(getattr(a, name), getattr(b, name)), name
+
+
+@pytest.mark.parametrize("T", [0.0, 1.0])
+def test_verify_step_reads_inputs_written_just_before_on_its_stream(cuda_lib, orc, T):
+    """Inputs written on the caller's stream right before eagle_verify_step, behind a kernel
+    that spins for about 10 ms, are the ones the step reads, the side stream's attention
+    included (it starts after the LM head, so after all earlier work on the caller's
+    stream).  The step's buffers hold NaN until the copies land."""
+    from tree_verify_b200.step import StepInputs, VerifyStep, shape_from_workload
+    base, kw = STEP_CASES["vicuna"]
+    w = wl.scaled(wl.WORKLOADS[base], **kw)
+    inp = wl.generate(w, T)
+    shape = shape_from_workload(w)
+    src = StepInputs.from_numpy(inp, w.dtype)
+    x = StepInputs.from_numpy(inp, w.dtype)
+    names = ("q", "k_prefix", "v_prefix", "k_tree", "v_tree", "hidden", "w_lm", "draft_probs")
+    for n in names:
+        getattr(x, n).fill_(float("nan"))
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    a, b = VerifyStep(shape), VerifyStep(shape)
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(20_000_000)
+        for n in names:
+            getattr(x, n).copy_(getattr(src, n))
+    a.run(x, T, 3, 4, stream=s)
+    torch.cuda.synchronize()
+    b.attention(src)
+    b.lm_head(src)
+    b.accept(src, T, 3, 4)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_error(reset=True) == 0
+    for name in ("logits", "accepted_nodes", "accept_len", "next_token"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    ref = orc.tree_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["prefix_lens"],
+                             inp["k_tree"], inp["v_tree"], inp["parents"])
+    got = a.out.float().cpu().numpy().reshape(-1, w.head_dim)
+    err = row_rel_err(got, ref.reshape(-1, w.head_dim))
+    assert err.max() <= TOL[w.dtype], f"attention max row error {err.max():.3e}"

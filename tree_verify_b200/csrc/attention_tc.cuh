@@ -27,12 +27,14 @@
 //                     its TMA tile), in the order PV(t), S(t + 2);
 //   warps 10-11       no role (a 384-thread block caps registers at 168, which three warps
 //                     per SM sub-partition can hold).
-// TMEM: two S buffers of 128 columns, then O (D columns).  S(t) goes to buffer t % 2, so
+// TMEM: three S buffers of 128 columns, then O (D columns).  S(t) goes to buffer t % 3, so
 // the tensor core computes S(t + 1) while the groups work on tile t; the bf16 P of each
-// half is written over the first 32 columns of that half of S(t).  The MMAs of one CTA run
-// in issue order, so S(t + 2), issued after PV(t), overwrites P(t) only once PV(t) has read
-// it.  The groups wait for PV(t - 1) (pv_done) before they rescale O, and before they
-// announce P(t), so they never run two barrier phases ahead of the MMA issuer.  O is
+// half is written over the first 32 columns of that half of S(t).  S(t + 2) is issued after
+// PV(t) into the buffer of S(t - 1) and P(t - 1), once the issuer has seen PV(t - 1)
+// complete (pv_done): the ordering rests on barriers, not on the order in which the
+// tensor core runs MMAs of different accumulators.  The groups wait for PV(t - 1) before
+// they rescale O, and before they announce P(t), so they never run two barrier phases
+// ahead of the MMA issuer.  O is
 // rescaled lazily (each group its half of the columns), only when the row maximum grows by
 // more than 2^8 over the reference the P values were taken against.  The last split also
 // runs the tree tile: its K/V rows come by TMA from a 4-D view of the tree K/V
@@ -75,13 +77,14 @@ struct TcSmem {
   static constexpr int kBarOff = kLOff + 2 * kTcRows * 4;
   // q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[buffer], p_full,
   // pv_done, o_final
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 1 + 1 + 1;
+  static constexpr int kSBufs = 3;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + kSBufs + 1 + 1 + 1;
   static constexpr int kBytes = kBarOff + kNumBars * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;
-  // TMEM columns: S(t) in buffer u = t % 2 at kSCol + kAttnKeys u (keys in column order;
-  // the P of group g over the kTcHalf / 2 columns from kTcHalf g), O at kOCol
+  // TMEM columns: S(t) in buffer u = t % kSBufs at kSCol + kAttnKeys u (keys in column
+  // order; the P of group g over the kTcHalf / 2 columns from kTcHalf g), O at kOCol
   static constexpr uint32_t kSCol = 0;
-  static constexpr uint32_t kOCol = 2 * kAttnKeys;
+  static constexpr uint32_t kOCol = kSBufs * kAttnKeys;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kOCol + D <= kTmemCols, "TMEM columns");
 };
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* v_full = k_empty + SK;
   uint64_t* v_empty = v_full + SV;
   uint64_t* s_full = v_empty + SV;  // [buffer]
-  uint64_t* p_full = s_full + 2;
+  uint64_t* p_full = s_full + SM::kSBufs;
   uint64_t* pv_done = p_full + 1;
   uint64_t* o_final = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_final + 1);
@@ -150,7 +153,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
     }
-    for (int u = 0; u < 2; ++u) mbar_init(smem_u32(&s_full[u]), 1);
+    for (int u = 0; u < SM::kSBufs; ++u) mbar_init(smem_u32(&s_full[u]), 1);
     mbar_init(smem_u32(p_full), kTcSoftmaxWarps);  // one arrival per softmax warp
     mbar_init(smem_u32(pv_done), 1);
     mbar_init(smem_u32(o_final), 1);
@@ -214,15 +217,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t idesc_s = idesc_bf16_f32(kTcRows, kAttnKeys);
       const uint32_t idesc_o = idesc_bf16_f32_bmn(kTcRows, D);
       bool ok = mbar_wait(smem_u32(q_full), 0, kErrAttnMmaWait);
-      // S(t) = Q K^T over the 128 keys of tile t, one M 128 x N 128 chain into buffer t % 2.
-      // That buffer last held S(t - 2) and P(t - 2): both groups arrived on p_full before
-      // PV(t - 2) was issued, and PV(t - 2) was issued before this chain.
+      // S(t) = Q K^T over the 128 keys of tile t, one M 128 x N 128 chain into buffer t % 3.
+      // That buffer last held S(t - 3) and P(t - 3): both groups arrived on p_full before
+      // PV(t - 3) was issued, and the issuer saw PV(t - 3) complete before it issued PV(t - 2),
+      // which precedes this chain.
       auto issue_s = [&](int t) {
         const int s = t % SK;
         ok = ok && mbar_wait(smem_u32(&k_full[s]), (t / SK) & 1, kErrAttnMmaWait);
         tc_fence_after();
         const uint32_t kb = k_stage(s);
-        const uint32_t d_tmem = tmem + SM::kSCol + static_cast<uint32_t>((t & 1) * kAttnKeys);
+        const uint32_t d_tmem = tmem + SM::kSCol + static_cast<uint32_t>((t % SM::kSBufs) * kAttnKeys);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int h = kk >> 2, k4 = kk & 3;
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t bdesc = smem_desc_k_sw128(kb + h * kAttnKeys * 128) + 2 * k4;
           if (ok) tc_mma_f16(d_tmem, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[t & 1]));
+        tc_commit(smem_u32(&s_full[t % SM::kSBufs]));
         tc_commit(smem_u32(&k_empty[s]));
       };
       // O += P V over the tile's 128 keys: 8 MMAs of 16 keys (8 TMEM columns of P from the
@@ -239,10 +243,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       auto issue_pv = [&](int t) {
         const int s = t % SV;
         ok = ok && mbar_wait(smem_u32(p_full), t & 1, kErrAttnMmaWait);
+        // PV(t - 1) complete: S(t + 2), issued next, may overwrite its P.  Waited for before
+        // this PV's commit, so the barrier is never two phases ahead of this wait.
+        if (t > 0) ok = ok && mbar_wait(smem_u32(pv_done), (t - 1) & 1, kErrAttnMmaWait);
         ok = ok && mbar_wait(smem_u32(&v_full[s]), (t / SV) & 1, kErrAttnMmaWait);
         tc_fence_after();
         const uint32_t vb = v_stage(s);
-        const uint32_t pa = tmem + SM::kSCol + static_cast<uint32_t>((t & 1) * kAttnKeys);
+        const uint32_t pa = tmem + SM::kSCol + static_cast<uint32_t>((t % SM::kSBufs) * kAttnKeys);
         const uint32_t o_tmem = tmem + SM::kOCol;
 #pragma unroll
         for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
@@ -298,10 +305,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float m_ref = -INFINITY, l = 0.f;
     for (int t = 0; t < T; ++t) {
       const bool tree = t >= nt;
-      mbar_wait(smem_u32(&s_full[t & 1]), (t >> 1) & 1, kErrAttnConsumerWait);
+      mbar_wait(smem_u32(&s_full[t % SM::kSBufs]), (t / SM::kSBufs) & 1, kErrAttnConsumerWait);
       tc_fence_after();
       // this group's half of S(t), and its P(t) over the half's first 32 columns
-      const uint32_t s_col = lane_base + SM::kSCol + static_cast<uint32_t>((t & 1) * kAttnKeys + grp * kTcHalf);
+      const uint32_t s_col =
+          lane_base + SM::kSCol + static_cast<uint32_t>((t % SM::kSBufs) * kAttnKeys + grp * kTcHalf);
       float tmax_half = -INFINITY;
       float x[kTcHalf];
       if (live) {

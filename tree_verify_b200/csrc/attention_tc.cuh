@@ -34,12 +34,12 @@
 // complete (pv_done): the ordering rests on barriers, not on the order in which the
 // tensor core runs MMAs of different accumulators.  The groups wait for PV(t - 1) before
 // they rescale O, and before they announce P(t), so they never run two barrier phases
-// ahead of the MMA issuer.  O is
-// rescaled lazily (each group its half of the columns), only when the row maximum grows by
-// more than 2^8 over the reference the P values were taken against.  The last split also
-// runs the tree tile: its K/V rows come by TMA from a 4-D view of the tree K/V
-// ([B][N][Hkv][D], rows past N zero-filled).  Splits write (m, l, acc) partials for the
-// log-sum-exp merge; a single split normalises and writes the output.
+// ahead of the MMA issuer.  O is rescaled lazily (each group its half of the columns),
+// only when the row maximum grows by more than 2^8 over the reference the P values were
+// taken against.  The last split also runs the tree tile: its K/V rows come by TMA from a
+// 4-D view of the tree K/V ([B][N][Hkv][D], rows past N zero-filled).  Splits write
+// (m, l, acc) partials for the log-sum-exp merge; a single split normalises and writes the
+// output.
 #pragma once
 
 #include "attention.cuh"
